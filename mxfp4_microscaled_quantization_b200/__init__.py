@@ -1,0 +1,10 @@
+"""B200-native MXFP4 attention with Universal Optimal Scaling and
+Pre-Normalization Quantization (MXAttention), behind a C-ABI CUDA library.
+
+The compute runs in ``libmxattn.so`` (CUDA kernels for sm_100a); this package
+only marshals arguments.  Importing it does not load the library; the first
+call does, and fails loudly if the library was not built.
+"""
+from . import workloads  # noqa: F401
+
+__all__ = ["workloads"]

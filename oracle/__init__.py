@@ -1,0 +1,175 @@
+"""CPU oracle for MXFP4 attention with UOS and PNQ (fp64, plain C loops).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg are the only callers.  The product path never
+imports this package.  It shares no code with the CUDA library; both take
+their inputs from ``mxfp4_microscaled_quantization_b200.workloads``.
+
+What each function computes, and the reading behind it, is documented beside
+the C code in ``oracle.c`` (source: the MXAttention abstract, "MXAttention:
+Data-Free Optimal Scaling and Pre-Normalization Quantization for MXFP4
+Attention").  Every function here is pinned by the ``-m "not gpu"`` tests
+(E2M1 grid and brute-force rounding, the OCP and UOS scale invariants,
+equivariance, exact online softmax, PNQ normalization, hand-derived golden
+cases); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+RULES = {"ocp": 0, "uos": 1, "none": 2}
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c with gcc (fp64, no fast-math, no FMA contraction, OpenMP over rows)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+               "-fno-fast-math", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        L.oracle_e2m1_encode_batch.argtypes = [P, i64, P]
+        L.oracle_scale_exponent_batch.argtypes = [P, i64, ctypes.c_int, P]
+        L.oracle_quantize_rows.argtypes = [P, i64, i64, ctypes.c_int, P, P]
+        L.oracle_quantize_cols.argtypes = [P, i64, i64, i64, ctypes.c_int, P, P]
+        L.oracle_dequantize_rows.argtypes = [P, P, i64, i64, P]
+        L.oracle_attention_head.argtypes = [P, P, P, i64, i64, i64, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_double, P, i64, P, ctypes.c_int]
+        L.oracle_attention_head.restype = ctypes.c_int
+        L.oracle_max_threads.restype = ctypes.c_int
+        L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e2m1_decode.restype = ctypes.c_double
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _rule(r) -> int:
+    return RULES[r] if isinstance(r, str) else int(r)
+
+
+def max_threads() -> int:
+    return int(lib().oracle_max_threads())
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    codes = np.asarray(codes, dtype=np.uint8)
+    return np.array([lib().oracle_e2m1_decode(int(c)) for c in codes.ravel()]).reshape(codes.shape)
+
+
+def e2m1_encode(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e2m1_encode_batch(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def scale_exponent(amax, rule) -> np.ndarray:
+    a = np.ascontiguousarray(amax, dtype=np.float64)
+    out = np.empty(a.shape, dtype=np.int32)
+    lib().oracle_scale_exponent_batch(_ptr(a), a.size, _rule(rule), _ptr(out))
+    return out
+
+
+def quantize_rows(x_bits: np.ndarray, rule):
+    """bf16 bits [rows, cols] -> (codes uint8 [rows, cols/2], scales uint8 [rows, cols/32])."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    cols = x.shape[-1]
+    assert cols % 32 == 0
+    rows = x.size // cols
+    codes = np.empty(x.shape[:-1] + (cols // 2,), dtype=np.uint8)
+    scales = np.empty(x.shape[:-1] + (cols // 32,), dtype=np.uint8)
+    lib().oracle_quantize_rows(_ptr(x), rows, cols, _rule(rule), _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def quantize_cols(v_bits: np.ndarray, rule):
+    """V bf16 bits [..., N, d] -> V^T (codes [..., d, Npad/2], scales [..., d, Npad/32])."""
+    v = np.ascontiguousarray(v_bits, dtype=np.uint16)
+    N, d = v.shape[-2:]
+    BH = v.size // (N * d)
+    npad = (N + 31) // 32 * 32
+    lead = v.shape[:-2]
+    codes = np.empty(lead + (d, npad // 2), dtype=np.uint8)
+    scales = np.empty(lead + (d, npad // 32), dtype=np.uint8)
+    lib().oracle_quantize_cols(_ptr(v), BH, N, d, _rule(rule), _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    cols = codes.shape[-1] * 2
+    rows = codes.size * 2 // cols
+    out = np.empty(codes.shape[:-1] + (cols,), dtype=np.float64)
+    lib().oracle_dequantize_rows(_ptr(codes), _ptr(scales), rows, cols, _ptr(out))
+    return out
+
+
+def attention(Q, K, V, kv_tile, rule="uos", pnq=True, p_rule=None, scale=None, rows=None, nthreads=0):
+    """MXFP4 attention forward on the CPU in fp64.
+
+    Q, K, V: bf16 bits [B, H, N, d].  `rule` quantizes Q, K, V (and P unless
+    `p_rule` says otherwise); "none" disables quantization.  `rows`: None for
+    all rows, else an int array of query rows (the same rows for every head)
+    or a list with one array per (b, h).  Returns fp64 [B, H, R, d].
+    """
+    Q = np.ascontiguousarray(Q, dtype=np.uint16)
+    K = np.ascontiguousarray(K, dtype=np.uint16)
+    V = np.ascontiguousarray(V, dtype=np.uint16)
+    B, H, N, d = Q.shape
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    in_rule = _rule(rule)
+    pr = in_rule if p_rule is None else _rule(p_rule)
+    per_head_rows = []
+    for bh in range(B * H):
+        if rows is None:
+            r = np.arange(N, dtype=np.int64)
+        elif isinstance(rows, (list, tuple)):
+            r = np.asarray(rows[bh], dtype=np.int64)
+        else:
+            r = np.asarray(rows, dtype=np.int64)
+        per_head_rows.append(np.ascontiguousarray(r))
+    R = len(per_head_rows[0])
+    assert all(len(r) == R for r in per_head_rows)
+    out = np.empty((B, H, R, d), dtype=np.float64)
+    Qf = Q.reshape(B * H, N, d)
+    Kf = K.reshape(B * H, N, d)
+    Vf = V.reshape(B * H, N, d)
+    ov = out.reshape(B * H, R, d)
+    for bh in range(B * H):
+        o = np.empty((R, d), dtype=np.float64)
+        st = lib().oracle_attention_head(_ptr(Qf[bh]), _ptr(Kf[bh]), _ptr(Vf[bh]), N, d, kv_tile, in_rule, pr,
+                                         1 if pnq else 0, float(scale), _ptr(per_head_rows[bh]), R, _ptr(o),
+                                         int(nthreads))
+        if st != 0:
+            raise RuntimeError(f"oracle_attention_head failed with status {st}")
+        ov[bh] = o
+    return out
