@@ -1,0 +1,367 @@
+"""Benchmark: MXFP4 attention with UOS + PNQ (MXAttention) on B200.
+
+One step = the whole hot path on one batch: Q/K and V^T quantize/pack
+(mxattn_prepare) + the fused attention kernel (mxattn_attend), i.e.
+mxattn_forward, on the video-DiT self-attention workload B=1, H=40,
+N=32760 (21 frames x 30 x 52 tokens), d=128, kv_tile=128, UOS + PNQ, with
+synthetic seeded inputs already resident in HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun (N > 1) every rank runs its own batch (seed = rank): weak
+scaling with no data-path collective; the timed region is bracketed by a
+barrier and synchronize, and the slowest rank's time counts.  Rank 0 prints
+one JSON line.  `--impl reference` times the CPU oracle (fp64, plain loops) on
+a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mxfp4_microscaled_quantization_b200 import workloads as wl  # noqa: E402
+
+METRIC = "MXFP4 attention TFLOPS (4BHN²d) and % of B200 FP4 peak at N=32760,d=128"
+UNIT = "TFLOP/s"
+WORKLOAD = wl.WORKLOADS["video_dit"]
+FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor ratio (9 : 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ATTN_PROFILE = os.path.join(ROOT, "profiles", "attention_video_dit.md")
+ATTN_SOURCE = os.path.join(ROOT, "mxfp4_microscaled_quantization_b200", "csrc", "attention.cu")
+
+
+def config_dict(w=WORKLOAD):
+    return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} ({w.frames}x{w.rows}x{w.cols} tokens) d={w.d} "
+                        f"kv_tile={w.kv_tile}, UOS + PNQ, smooth low-rank + noise bf16 inputs",
+            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "kv_tile": w.kv_tile, "rule": "uos", "pnq": True,
+            "step": "mxattn_prepare (Q/K + V^T quantize) + mxattn_attend (fused attention)",
+            "l2": "inputs larger than L2: 1.0 GB of bf16 Q/K/V per step (no flush)"}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profiled_traffic():
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu
+    summary, if it was taken on the current attention.cu; else None."""
+    try:
+        with open(ATTN_PROFILE) as f:
+            text = f.read()
+        with open(ATTN_SOURCE, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    src = [ln for ln in text.splitlines() if ln.startswith("source_sha256_16:")]
+    tr = [ln for ln in text.splitlines() if ln.startswith("dram_bytes_per_full_launch:")]
+    if not src or not tr or src[0].split(":", 1)[1].strip() != digest:
+        return None
+    return float(tr[0].split(":", 1)[1].strip())
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"mxattn_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "200"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        loaded = [s for s in sm if smax and s >= 0.3 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons, "samples": len(rows)}
+
+
+def oracle_sample(Q, K, V, w, rows, nthreads=0):
+    """The CPU oracle on `rows` query rows of head 0 (plus its K/V quantization)."""
+    import oracle
+
+    t0 = time.perf_counter()
+    oracle.attention(Q[:, :1], K[:, :1], V[:, :1], w.kv_tile, rule="uos", pnq=True, rows=rows, nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(Q, K, V, w, budget_s=15.0):
+    """Time the oracle as it stands on a bounded sample: query rows of head 0 sized to
+    about `budget_s` of CPU work, converted to the same unit (4*N*d flops per row)."""
+    import oracle
+
+    threads = oracle.max_threads()
+    probe = np.arange(0, w.N, max(1, w.N // (2 * threads)))[: 2 * threads]
+    t = oracle_sample(Q, K, V, w, probe, threads)
+    per_row = t / len(probe)
+    n = int(min(w.N, max(len(probe), budget_s / max(per_row, 1e-9))))
+    rows = np.linspace(0, w.N - 1, n).astype(np.int64)
+    t = oracle_sample(Q, K, V, w, rows, threads)
+    flops = 4.0 * n * w.N * w.d
+    return {"value": flops / t / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n} query rows of head 0 of {w.name} (full K/V quantization of that head included), "
+                      f"{t:.1f} s on {threads} OpenMP threads"}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle on the host cores (rank 0 only)."""
+    if rank != 0:
+        return 0
+    import oracle
+
+    w = WORKLOAD
+    Q, K, V = wl.make_qkv(w, seed=0)
+    threads = oracle.max_threads()
+    # size one step to a bounded sample so warmup + steps stay within a few minutes
+    probe = np.arange(threads) * (w.N // threads)
+    per_row = oracle_sample(Q, K, V, w, probe, threads) / len(probe)
+    step_budget_s = max(2.0, 120.0 / (args.warmup + args.steps))  # whole run within a few minutes
+    n = int(max(threads, min(w.N, step_budget_s / max(per_row, 1e-9))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        rng = np.random.default_rng(i)
+        rows = np.sort(rng.choice(w.N, n, replace=False))
+        t = oracle_sample(Q, K, V, w, rows, threads)
+        if i >= args.warmup:
+            times.append(t)
+    t_step = sum(times) / len(times)
+    value = 4.0 * n * w.N * w.d / t_step / 1e12
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": config_dict(),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"per step {n} seeded query rows of head 0 (with that head's K/V "
+                                       f"quantization) on {threads} OpenMP threads"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def quantize_sweep_point(torch, mx, peaks, peak_kind, log2n=30, iters=10):
+    """Standalone quantize kernel on the largest quantize-sweep size (2^30 bf16 elements)."""
+    x = wl.student_t_matrix(1 << log2n, 4096, seed=0)
+    xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    del x
+    codes = torch.empty((xd.shape[0], 2048), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((xd.shape[0], 128), dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        mx.mxattn_quantize(xd, "uos", codes, scales)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        mx.mxattn_quantize(xd, "uos", codes, scales)
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / iters
+    nbytes = (1 << log2n) * (2 + 0.5 + 1 / 32)
+    gbs = nbytes / t / 1e9
+    out = {"elements": 1 << log2n, "bytes_per_element": 2.53125, "us_per_launch": t * 1e6, "achieved_gbs": gbs,
+           "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
+           "frac_of_8tbs_spec": gbs / 8000.0, "peak_kind": peak_kind, "rule": "uos"}
+    del xd, codes, scales
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+
+    from mxfp4_microscaled_quantization_b200 import mxattn as mx
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    w = WORKLOAD
+    peaks, peak_kind = load_peaks()
+    B, H, N, d = w.B, w.H, w.N, w.d
+
+    Q, K, V = wl.make_qkv(w, seed=rank)
+    base = None
+    if rank == 0:
+        base = cpu_baseline(Q, K, V, w, budget_s=args.cpu_budget)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)  # noqa: E731
+    q, k, v = to_dev(Q), to_dev(K), to_dev(V)
+    out = torch.empty((B, H, N, d), dtype=torch.float32, device="cuda")
+    ws = mx.new_workspace(B, H, N, d)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        mx.mxattn_prepare(q, k, v, "uos", ws)
+        if ev is not None:
+            ev[1].record(stream)
+        mx.mxattn_attend(ws, B, H, N, d, w.kv_tile, True, "uos", 0.0, out)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if mx.mxattn_workspace_status(ws) != 0:
+        raise RuntimeError("attention kernel reported a timeout during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            step(evs[i])
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    total_ms = evs[0][0].elapsed_time(evs[-1][2])
+    attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    prep_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    if mx.mxattn_workspace_status(ws) != 0:
+        raise RuntimeError("attention kernel reported a timeout")
+    t = torch.tensor([total_ms, sum(attn_ms) / len(attn_ms)], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, attn_avg_ms = float(t[0]), float(t[1])
+    ms_per_step = total_ms / args.steps
+    value = world * w.flops / (ms_per_step / 1e3) / 1e12
+
+    # end to end through the public API with host buffers (pinned), H2D + D2H inside the timed region
+    q_h = torch.from_numpy(Q.view(np.int16)).view(torch.bfloat16).pin_memory()
+    k_h = torch.from_numpy(K.view(np.int16)).view(torch.bfloat16).pin_memory()
+    v_h = torch.from_numpy(V.view(np.int16)).view(torch.bfloat16).pin_memory()
+    o_h = torch.empty((B, H, N, d), dtype=torch.float32).pin_memory()
+    bufs = (q, k, v, out, ws)
+    for _ in range(2):
+        mx.attention_from_host(q_h, k_h, v_h, w.kv_tile, True, "uos", 0.0, bufs, o_h)
+    torch.cuda.synchronize()
+    e2e_steps = max(2, min(args.steps, 5))
+    if dist is not None:
+        dist.barrier()
+    ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ee0.record(stream)
+    for _ in range(e2e_steps):
+        mx.attention_from_host(q_h, k_h, v_h, w.kv_tile, True, "uos", 0.0, bufs, o_h)
+    ee1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([ee0.elapsed_time(ee1) / e2e_steps], dtype=torch.float64, device="cuda")
+    if dist is not None:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te[0])
+
+    quant = None
+    if rank == 0 and not args.no_quantize_sweep:
+        quant = quantize_sweep_point(torch, mx, peaks, peak_kind)
+
+    if rank == 0:
+        attn_tflops = w.flops / (attn_avg_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
+        clocks = clk.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "mxfp4 (e2m1 x e8m0, fp32 accumulate)", "data": "synthetic",
+            "config": {**config_dict(), "parallelism": f"{world} independent replicas (one batch per rank)"},
+            "pct_of_fp4_peak": 100.0 * value / world / peak,
+            "roofline": {"bound": "tensor", "kernel": "mxattn_fwd_kernel<128,128>", "achieved": attn_tflops,
+                         "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                         "traffic": profiled_traffic(),
+                         "peak_source": f"{peak_kind} bf16 sustained {peaks['bf16_tflops_sustained']} TFLOP/s x "
+                                        f"{FP4_PER_BF16:g} (nominal dense fp4:bf16)",
+                         "attn_ms": attn_avg_ms, "prepare_ms": sum(prep_ms) / len(prep_ms),
+                         "frac_of_9pf_spec": attn_tflops / 9000.0},
+            "cpu_baseline": base,
+            "e2e": {"value": world * w.flops / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+                    "h2d_bytes_per_step": 3 * B * H * N * d * 2, "d2h_bytes_per_step": B * H * N * d * 4,
+                    "ms_per_step": e2e_ms, "api": "attention_from_host -> mxattn_forward"},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks,
+            "quantize_sweep": quant,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-quantize-sweep", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    args.warmup = max(args.warmup, 3)  # timing rule: at least 3 warm-up steps
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_gpu(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

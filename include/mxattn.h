@@ -1,0 +1,166 @@
+/*
+ * mxattn.h -- C ABI of libmxattn.so: MXFP4 attention with Universal Optimal
+ * Scaling (UOS) and Pre-Normalization Quantization (PNQ) on NVIDIA B200
+ * (sm_100a).
+ *
+ * Method: "MXAttention: Data-Free Optimal Scaling and Pre-Normalization
+ * Quantization for MXFP4 Attention", abstract.  It fixes the MXFP4 operand
+ * format ("OCP MXFP4", power-of-two microscaling), the UOS scaling boundary
+ * Qmax = 7.25, and PNQ: the unnormalized softmax exponentials are quantized
+ * before the row-wise sum, so the sum is built from the same quantized values
+ * that weight V.  Readings of what the abstract leaves open:
+ *   - MXFP4 blocks are 32 consecutive elements along the contraction axis of
+ *     each product (Q, K: along the head dimension d; P: along keys, aligned
+ *     to key-tile starts; V: along tokens), with E2M1 elements
+ *     {0, .5, 1, 1.5, 2, 3, 4, 6} x sign and one E8M0 scale 2^e per block.
+ *   - OCP rule: e = floor(log2 amax) - 2.  UOS rule: the smallest e with
+ *     amax <= 7.25 * 2^e.  Both clamp e to [-127, 127]; amax = 0 gives -127.
+ *   - Elements round to nearest, ties to the even code, saturating at 6; the
+ *     sign of a value that rounds to zero is kept (code 0x8).
+ *   - The softmax scale is applied to the fp32 product of the dequantized Q
+ *     and K; the online softmax walks key tiles of kv_tile columns in
+ *     ascending order and subtracts the running maximum after each tile.
+ *   - PNQ off: P*V still uses the quantized exponentials but the row sum uses
+ *     the unquantized ones (the abstract's "row-wise normalization error").
+ *
+ * Conventions for every entry point:
+ *   - Pointers are device pointers unless stated otherwise; the caller owns
+ *     every buffer, including the workspace.  The library allocates no device
+ *     memory and keeps no state between calls except cached function handles.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Argument errors are returned synchronously and launch
+ *     nothing.  MXATTN_ERR_CUDA reports a launch error (cudaGetLastError).
+ *   - Layouts are row-major and contiguous.  A code byte holds element 2i in
+ *     its low nibble and element 2i+1 in its high nibble.  A scale byte is
+ *     the E8M0 encoding e + 127.
+ *   - bf16 inputs are IEEE bfloat16 bit patterns; NaN and Inf inputs are
+ *     outside the contract (the result is unspecified but the call is safe).
+ */
+#ifndef MXATTN_H
+#define MXATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* mxattn_stream_t;
+
+typedef enum {
+    MXATTN_OK = 0,
+    MXATTN_ERR_INVALID = 1,     /* null pointer, negative or inconsistent size, small workspace */
+    MXATTN_ERR_UNSUPPORTED = 2, /* d or kv_tile outside the supported set, N too large */
+    MXATTN_ERR_CUDA = 3,        /* a CUDA launch or driver call failed */
+    MXATTN_ERR_TIMEOUT = 4      /* a bounded wait inside the attention kernel gave up (read via
+                                   mxattn_workspace_status) */
+} mxattn_status;
+
+typedef enum {
+    MXATTN_RULE_OCP = 0, /* e = floor(log2 amax) - 2 */
+    MXATTN_RULE_UOS = 1  /* smallest e with amax <= 7.25 * 2^e (abstract: "Qmax=7.25") */
+} mxattn_rule;
+
+/*
+ * Standalone MXFP4 quantize/pack (the abstract's "direct MXFP4 quantization";
+ * the scale rule is UOS or OCP).
+ *   x:      bf16 [rows, cols], cols % 32 == 0, 16-byte aligned.
+ *   codes:  u8 [rows, cols/2] (packed E2M1), 4-byte aligned.
+ *   scales: u8 [rows, cols/32] (E8M0), one per 32-element block.
+ * rows == 0 is a no-op.  Errors: MXATTN_ERR_INVALID for null pointers,
+ * negative sizes, cols % 32 != 0 or misaligned pointers.
+ */
+mxattn_status mxattn_quantize(const void* x, int64_t rows, int64_t cols, mxattn_rule rule,
+                              uint8_t* codes, uint8_t* scales, mxattn_stream_t stream);
+
+/*
+ * V quantize with transpose: blocks of 32 consecutive tokens of each channel
+ * (reading: the scale runs along the contraction axis of P*V).
+ *   v:        bf16 [BH, N, d], d in {64, 128}, 16-byte aligned.
+ *   codes_t:  u8 [BH, d, Npad/2], Npad = ceil(N/32)*32; tokens >= N are zeros.
+ *   scales_t: u8 [BH, d, Npad/32].
+ * Errors: MXATTN_ERR_INVALID (null, N < 1, BH < 1), MXATTN_ERR_UNSUPPORTED (d).
+ */
+mxattn_status mxattn_quantize_vt(const void* v, int64_t BH, int64_t N, int64_t d, mxattn_rule rule,
+                                 uint8_t* codes_t, uint8_t* scales_t, mxattn_stream_t stream);
+
+/*
+ * Bytes of workspace that mxattn_forward / mxattn_forward_quantized need for
+ * this shape (0 for invalid shapes).  With G = ceil(N/128), Npad =
+ * ceil(N/32)*32 and every region starting on a 256-byte boundary, the
+ * workspace holds, in order:
+ *   status   256 bytes (u32 error word of the last forward on this workspace)
+ *   q_codes  B*H*N*d/2      k_codes  B*H*N*d/2      vt_codes B*H*d*Npad/2
+ *   q_sf     B*H*G*512      k_sf     B*H*G*512      vt_sf    B*H*G*512
+ * The *_codes regions use the layouts of mxattn_quantize / mxattn_quantize_vt.
+ * The *_sf regions hold the E8M0 scales regrouped per 128 rows (Q, K) or 128
+ * tokens (V^T): within a group, row m (or channel m of V^T) and block k sit at
+ * byte (m%32)*16 + (m/32)*4 + k -- the order in which the tensor core reads
+ * scale factors -- with rows past N set to 0 and unused V^T channel rows to
+ * 127.
+ */
+size_t mxattn_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Fused MXFP4 attention forward, non-causal:
+ *   O = softmax(deq(Qq) deq(Kq)^T * softmax_scale) with MXFP4 P, times deq(Vq),
+ * evaluated as the tile-ordered online softmax described above.
+ *   Q, K, V: bf16 [B, H, N, d], 16-byte aligned.  O: fp32 [B, H, N, d], 16-byte aligned.
+ *   d in {64, 128}; kv_tile in {64, 128}; 1 <= N <= 2^24; pnq in {0, 1};
+ *   rule applies to Q, K, V and P; softmax_scale <= 0 selects 1/sqrt(d).
+ *   workspace: >= mxattn_workspace_size(B, H, N, d) bytes, 256-byte aligned.
+ * Launches three kernels on `stream`: Q/K quantize, V^T quantize, attention.
+ * The attention kernel's waits are bounded; if one gives up it records
+ * MXATTN_ERR_TIMEOUT in the workspace status word (see
+ * mxattn_workspace_status) and O is unspecified.
+ */
+mxattn_status mxattn_forward(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                             int kv_tile, int pnq, mxattn_rule rule, float softmax_scale, float* O,
+                             void* workspace, size_t workspace_bytes, mxattn_stream_t stream);
+
+/*
+ * mxattn_forward in two calls, for callers that time or schedule the steps
+ * separately: mxattn_prepare launches the Q/K and V^T quantize kernels into
+ * the workspace (and resets its status word); mxattn_attend launches the
+ * attention kernel on a workspace that mxattn_prepare filled for the same
+ * (B, H, N, d) and `rule`.  mxattn_forward == mxattn_prepare + mxattn_attend.
+ * Same constraints and errors as mxattn_forward.
+ */
+mxattn_status mxattn_prepare(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                             mxattn_rule rule, void* workspace, size_t workspace_bytes, mxattn_stream_t stream);
+mxattn_status mxattn_attend(int B, int H, int N, int d, int kv_tile, int pnq, mxattn_rule rule, float softmax_scale,
+                            float* O, void* workspace, size_t workspace_bytes, mxattn_stream_t stream);
+
+/*
+ * The attention step alone, on operands already quantized by the caller in
+ * the public layouts: q_codes/k_codes u8 [B,H,N,d/2], q_scales/k_scales u8
+ * [B,H,N,d/32] (as mxattn_quantize), vt_codes u8 [B,H,d,Npad/2], vt_scales u8
+ * [B,H,d,Npad/32] (as mxattn_quantize_vt).  `rule` is the rule for P.  The
+ * scales are regrouped into the workspace's *_sf regions first (the codes
+ * regions of the workspace are not used).  Same constraints and errors as
+ * mxattn_forward; code pointers 16-byte aligned.
+ */
+mxattn_status mxattn_forward_quantized(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
+                                       const uint8_t* k_scales, const uint8_t* vt_codes, const uint8_t* vt_scales,
+                                       int B, int H, int N, int d, int kv_tile, int pnq, mxattn_rule rule,
+                                       float softmax_scale, float* O, void* workspace, size_t workspace_bytes,
+                                       mxattn_stream_t stream);
+
+/*
+ * Synchronizes `stream`, reads the status word of `workspace` (written by
+ * the last forward that used it) and returns MXATTN_OK or
+ * MXATTN_ERR_TIMEOUT.  MXATTN_ERR_CUDA if the synchronization or copy fails.
+ * The word is reset by the next forward on this workspace.
+ */
+mxattn_status mxattn_workspace_status(const void* workspace, mxattn_stream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* mxattn_status_string(mxattn_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXATTN_H */

@@ -6,5 +6,19 @@ only marshals arguments.  Importing it does not load the library; the first
 call does, and fails loudly if the library was not built.
 """
 from . import workloads  # noqa: F401
-
-__all__ = ["workloads"]
+from .mxattn import (  # noqa: F401
+    MxattnError,
+    attention_from_host,
+    declared_symbols,
+    mxattn_attend,
+    mxattn_forward,
+    mxattn_forward_quantized,
+    mxattn_prepare,
+    mxattn_quantize,
+    mxattn_quantize_vt,
+    mxattn_status_string,
+    mxattn_workspace_size,
+    mxattn_workspace_status,
+    new_workspace,
+    workspace_layout,
+)

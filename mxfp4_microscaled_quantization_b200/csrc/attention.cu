@@ -1,0 +1,513 @@
+// attention.cu -- fused MXFP4 attention forward with UOS and PNQ for sm_100a.
+//
+// Method: "MXAttention: Data-Free Optimal Scaling and Pre-Normalization
+// Quantization for MXFP4 Attention", abstract: MXFP4 attention whose softmax
+// loop quantizes the unnormalized exponentials exp(S - m) of each key tile to
+// MXFP4 (scale rule UOS, Qmax = 7.25, or OCP) before the row sum, so the sum
+// is built from the same quantized values that weight V (PNQ).
+//
+// One CTA owns 128 query rows of one (batch, head) and walks all key tiles in
+// ascending order.  Roles (192 threads):
+//   warp 4 (one lane)  TMA producer: Q tile + scales once, then K and V^T
+//                      tiles (+ scales) into a kStages-deep ring.
+//   warp 5 (one lane)  MMA issuer: tcgen05.cp of E8M0 scales into TMEM and
+//                      tcgen05.mma kind::mxf4 block_scale for S = Q K^T
+//                      (double-buffered in TMEM) and O += P V.
+//   warps 0-3          softmax, one thread per query row (= TMEM lane):
+//                      running max, exp2 on the MUFU, per-32-column block
+//                      exponent (UOS/OCP), E2M1 packing of P into shared
+//                      memory, O rescale in TMEM when the max moved, and the
+//                      final O / l.
+// The row sum under PNQ is produced by the tensor core itself: V^T gets one
+// extra row of ones (E2M1 1.0, scale 2^0) so O's column d accumulates
+// sum_j q_j -- exactly the quantized values that multiply V -- and is
+// rescaled together with O.  Without PNQ the row sum of the unquantized
+// exponentials is kept in a register.
+//
+// Every mbarrier wait is bounded (kTimeoutNs); a wait that gives up records
+// MXATTN_ERR_TIMEOUT in the status word, raises a CTA-wide abort flag, and
+// every role drains its in-flight copies / MMAs before the CTA frees TMEM.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace mxattn {
+
+namespace {
+
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
+constexpr uint32_t kTimeoutCode = 4u;           // MXATTN_ERR_TIMEOUT
+
+template <int D, int T>
+struct Cfg {
+    static constexpr int kStages = 4;
+    static constexpr int kThreads = 192;
+    static constexpr int kQBytes = 128 * D / 2;
+    static constexpr int kKBytes = T * D / 2;
+    static constexpr int kVRows = D + 16;  // V^T rows + a row of ones + 15 zero rows
+    static constexpr int kVLoadBytes = D * T / 2;
+    static constexpr int kVStride = ((kVRows * T / 2) + 1023) / 1024 * 1024;
+    static constexpr int kPBytes = 128 * T / 2;
+    static constexpr int kSfBytes = 512;
+
+    static constexpr uint32_t kQKLayout = (D == 128) ? kLayoutSw64 : kLayoutSw32;
+    static constexpr uint32_t kQKSbo = 8 * D / 2;
+    static constexpr uint32_t kPVLayout = (T == 128) ? kLayoutSw64 : kLayoutSw32;
+    static constexpr uint32_t kPVSbo = 8 * T / 2;
+
+    // shared memory (offsets from a 1024-aligned base)
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kOffV = kOffK + kStages * kKBytes;
+    static constexpr int kOffP = kOffV + kStages * kVStride;
+    static constexpr int kOffQsf = kOffP + kPBytes;
+    static constexpr int kOffKsf = kOffQsf + kSfBytes;
+    static constexpr int kOffVsf = kOffKsf + kStages * kSfBytes;
+    static constexpr int kOffPsf = kOffVsf + kStages * kSfBytes;
+    static constexpr int kOffVsfConst = kOffPsf + kSfBytes;
+    static constexpr int kOffBar = kOffVsfConst + kSfBytes;
+    // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_empty[2], p_full, o_done, drain
+    static constexpr int kNumBars = 1 + 4 * kStages + 4 + 3;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kSmemUsed = kOffMisc + 16;
+    // >= 116 KB keeps one CTA per SM, so the 512-column TMEM allocation never waits
+    static constexpr int kSmemBytes = (kSmemUsed + 1024 > 116 * 1024) ? kSmemUsed + 1024 : 116 * 1024;
+
+    // TMEM columns
+    static constexpr uint32_t kColS0 = 0;
+    static constexpr uint32_t kColS1 = T;
+    static constexpr uint32_t kColO = 2 * T;
+    static constexpr uint32_t kColQsf = (2 * T + D + 16 + 3) / 4 * 4;
+    static constexpr uint32_t kColKsf = kColQsf + 4;
+    static constexpr uint32_t kColPsf = kColKsf + 4 * kStages;
+    static constexpr uint32_t kColVsf = kColPsf + 4;
+    static constexpr uint32_t kColsUsed = kColVsf + 8 * kStages;
+    static_assert(kColsUsed <= 512, "TMEM budget");
+};
+
+struct KParams {
+    const uint8_t* q_sf;
+    const uint8_t* k_sf;
+    const uint8_t* v_sf;
+    float* O;
+    uint32_t* status;
+    int N;
+    int ntq;     // query tiles per head
+    int nkv;     // key tiles per head
+    int groups;  // 128-row scale groups per head
+    int pnq;
+    int uos;
+    float kq;    // softmax_scale * log2(e)
+};
+
+__device__ __forceinline__ uint64_t sf_desc(const void* p) {
+    // 32 rows x 16 bytes, rows contiguous: core matrices of 8 rows 128 bytes apart
+    return smem_desc(smem_u32(p), 0, 128, kLayoutNone);
+}
+
+template <int D, int T>
+__global__ void __launch_bounds__(192, 1)
+    mxattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const KParams p) {
+    using C = Cfg<D, T>;
+    constexpr int S = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    uint8_t* sQ = smem + C::kOffQ;
+    uint8_t* sK = smem + C::kOffK;
+    uint8_t* sV = smem + C::kOffV;
+    uint8_t* sP = smem + C::kOffP;
+    uint8_t* sQsf = smem + C::kOffQsf;
+    uint8_t* sKsf = smem + C::kOffKsf;
+    uint8_t* sVsf = smem + C::kOffVsf;
+    uint8_t* sPsf = smem + C::kOffPsf;
+    uint8_t* sVsfConst = smem + C::kOffVsfConst;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    uint64_t* bar_q = bars;
+    uint64_t* bar_k_full = bars + 1;
+    uint64_t* bar_k_empty = bar_k_full + S;
+    uint64_t* bar_v_full = bar_k_empty + S;
+    uint64_t* bar_v_empty = bar_v_full + S;
+    uint64_t* bar_s_full = bar_v_empty + S;
+    uint64_t* bar_s_empty = bar_s_full + 2;
+    uint64_t* bar_p_full = bar_s_empty + 2;
+    uint64_t* bar_o_done = bar_p_full + 1;
+    uint64_t* bar_drain = bar_o_done + 1;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int bh = blockIdx.x / p.ntq;
+    const int qt = blockIdx.x % p.ntq;
+    const int nkv = p.nkv;
+
+    if (tid == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(bar_k_full + s, 1);
+            mbar_init(bar_k_empty + s, 1);
+            mbar_init(bar_v_full + s, 1);
+            mbar_init(bar_v_empty + s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_s_full + b, 1);
+            mbar_init(bar_s_empty + b, 128);
+        }
+        mbar_init(bar_p_full, 128);
+        mbar_init(bar_o_done, 1);
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    // Constant rows of every V^T stage: row D = ones (E2M1 1.0 = code 2), rows D+1.. = 0.
+    for (int idx = tid; idx < S * 16 * (T / 2) / 4; idx += C::kThreads) {
+        const int s = idx / (16 * (T / 2) / 4);
+        const int w = idx % (16 * (T / 2) / 4);
+        const int row = D + w / (T / 8);
+        reinterpret_cast<uint32_t*>(sV + s * C::kVStride + D * (T / 2))[w] = (row == D) ? 0x22222222u : 0u;
+    }
+    // Scale factors of V^T rows 128..255 (only used when D = 128): all 2^0.
+    for (int idx = tid; idx < 128; idx += C::kThreads) reinterpret_cast<uint32_t*>(sVsfConst)[idx] = 0x7F7F7F7Fu;
+    fence_proxy_async_smem();
+    if (warp == 5) {
+        tmem_alloc(tmem_holder, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tbase = *tmem_holder;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int k_issued = 0, v_issued = 0;
+            mbar_arrive_expect_tx(bar_q, C::kQBytes + C::kSfBytes);
+            tma_load_3d(sQ, &tmQ, bar_q, 0, qt * 128, bh);
+            bulk_load(sQsf, p.q_sf + (static_cast<size_t>(bh) * p.groups + qt) * 512, 512, bar_q);
+            for (int j = 0; j < nkv; ++j) {
+                const int s = j % S;
+                const uint32_t n = j / S;
+                const size_t grp = static_cast<size_t>(bh) * p.groups + (j * T) / 128;
+                if (j >= S && !mbar_wait_bounded(bar_k_empty + s, (n - 1) & 1, abort_flag, p.status, kTimeoutCode,
+                                                 kTimeoutNs))
+                    break;
+                mbar_arrive_expect_tx(bar_k_full + s, C::kKBytes + C::kSfBytes);
+                tma_load_3d(sK + s * C::kKBytes, &tmK, bar_k_full + s, 0, j * T, bh);
+                bulk_load(sKsf + s * 512, p.k_sf + grp * 512, 512, bar_k_full + s);
+                k_issued = j + 1;
+                if (j >= S && !mbar_wait_bounded(bar_v_empty + s, (n - 1) & 1, abort_flag, p.status, kTimeoutCode,
+                                                 kTimeoutNs))
+                    break;
+                mbar_arrive_expect_tx(bar_v_full + s, C::kVLoadBytes + C::kSfBytes);
+                tma_load_3d(sV + s * C::kVStride, &tmV, bar_v_full + s, j * (T / 2), 0, bh);
+                bulk_load(sVsf + s * 512, p.v_sf + grp * 512, 512, bar_v_full + s);
+                v_issued = j + 1;
+            }
+            // Drain: every copy this thread issued must land before the CTA exits.
+            // On the normal path these phases completed long ago and the waits return at once.
+            {
+                int dummy = 0;
+                volatile int* no_abort = &dummy;
+                mbar_wait_bounded(bar_q, 0, no_abort, p.status, kTimeoutCode, kTimeoutNs);
+                // only the newest tile of each stage can still be in flight
+                for (int j = k_issued - S < 0 ? 0 : k_issued - S; j < k_issued; ++j)
+                    mbar_wait_bounded(bar_k_full + j % S, (j / S) & 1, no_abort, p.status, kTimeoutCode, kTimeoutNs);
+                for (int j = v_issued - S < 0 ? 0 : v_issued - S; j < v_issued; ++j)
+                    mbar_wait_bounded(bar_v_full + j % S, (j / S) & 1, no_abort, p.status, kTimeoutCode, kTimeoutNs);
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t t_s[2] = {tbase + C::kColS0, tbase + C::kColS1};
+            const uint32_t t_o = tbase + C::kColO;
+            const uint64_t qdesc = smem_desc(smem_u32(sQ), 16, C::kQKSbo, C::kQKLayout);
+            const uint64_t pdesc = smem_desc(smem_u32(sP), 16, C::kPVSbo, C::kPVLayout);
+            bool ok = mbar_wait_bounded(bar_q, 0, abort_flag, p.status, kTimeoutCode, kTimeoutNs);
+            if (ok) {
+                tc_fence_after_sync();
+                tc_cp_sf(tbase + C::kColQsf, sf_desc(sQsf));
+                if (D == 128)
+                    for (int s = 0; s < S; ++s) tc_cp_sf(tbase + C::kColVsf + 8 * s + 4, sf_desc(sVsfConst));
+            }
+            auto issue_s = [&](int j) -> bool {
+                const int s = j % S;
+                const uint32_t n = j / S;
+                const int b = j & 1;
+                if (!mbar_wait_bounded(bar_k_full + s, n & 1, abort_flag, p.status, kTimeoutCode, kTimeoutNs))
+                    return false;
+                if (j >= 2 && !mbar_wait_bounded(bar_s_empty + b, ((j - 2) >> 1) & 1, abort_flag, p.status,
+                                                 kTimeoutCode, kTimeoutNs))
+                    return false;
+                tc_fence_after_sync();
+                tc_cp_sf(tbase + C::kColKsf + 4 * s, sf_desc(sKsf + s * 512));
+                const uint64_t kdesc = smem_desc(smem_u32(sK + s * C::kKBytes), 16, C::kQKSbo, C::kQKLayout);
+                const uint32_t ksf = tbase + C::kColKsf + 4 * s + ((T == 64) ? 2 * (j & 1) : 0);
+#pragma unroll
+                for (int kk = 0; kk < D / 64; ++kk)
+                    tc_mma_mxf4(t_s[b], qdesc + 2 * kk, kdesc + 2 * kk, mxf4_idesc(T, 2 * kk, 2 * kk),
+                                tbase + C::kColQsf, ksf, kk > 0 ? 1u : 0u);
+                tc_commit(bar_s_full + b);
+                tc_commit(bar_k_empty + s);
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            for (int j = 0; ok && j < nkv; ++j) {
+                if (j + 1 < nkv && !issue_s(j + 1)) break;
+                const int s = j % S;
+                const uint32_t n = j / S;
+                if (!mbar_wait_bounded(bar_p_full, j & 1, abort_flag, p.status, kTimeoutCode, kTimeoutNs)) break;
+                if (!mbar_wait_bounded(bar_v_full + s, n & 1, abort_flag, p.status, kTimeoutCode, kTimeoutNs))
+                    break;
+                tc_fence_after_sync();
+                tc_cp_sf(tbase + C::kColPsf, sf_desc(sPsf));
+                tc_cp_sf(tbase + C::kColVsf + 8 * s, sf_desc(sVsf + s * 512));
+                const uint64_t vdesc = smem_desc(smem_u32(sV + s * C::kVStride), 16, C::kPVSbo, C::kPVLayout);
+#pragma unroll
+                for (int kk = 0; kk < T / 64; ++kk) {
+                    const uint32_t sfb_id = (T == 64) ? 2u * (j & 1) : 2u * kk;
+                    tc_mma_mxf4(t_o, pdesc + 2 * kk, vdesc + 2 * kk, mxf4_idesc(D + 16, 2 * kk, sfb_id),
+                                tbase + C::kColPsf, tbase + C::kColVsf + 8 * s, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(bar_v_empty + s);
+                tc_commit(bar_o_done);
+            }
+            // Drain: wait for every MMA / copy this thread issued before TMEM is freed.
+            tc_commit(bar_drain);
+            int dummy = 0;
+            mbar_wait_bounded(bar_drain, 0, &dummy, p.status, kTimeoutCode, kTimeoutNs);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax (thread = query row)
+        const int row = tid;  // 0..127 == TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const float kq = p.kq;
+        const int uos = p.uos;
+        const int pnq = p.pnq;
+        const int valid_last = p.N - (nkv - 1) * T;
+        float m_run = -INFINITY;
+        float l_run = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nkv; ++j) {
+            const int b = j & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_s_full + b, (j >> 1) & 1, abort_flag, p.status,
+                                                            kTimeoutCode, kTimeoutNs))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+            float sv[T];
+#pragma unroll
+            for (int c = 0; c < T / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32_sync(tbase + lane_base + (b ? C::kColS1 : C::kColS0) + 32 * c, r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sv[32 * c + i] = __uint_as_float(r[i]);
+            }
+            tc_fence_before_sync();
+            mbar_arrive(bar_s_empty + b);
+            if (j == nkv - 1 && valid_last < T) {
+#pragma unroll
+                for (int i = 0; i < T; ++i)
+                    if (i >= valid_last) sv[i] = -INFINITY;
+            }
+            float bm[T / 32];
+#pragma unroll
+            for (int k = 0; k < T / 32; ++k) {
+                float a = sv[32 * k];
+#pragma unroll
+                for (int i = 1; i < 32; ++i) a = fmaxf(a, sv[32 * k + i]);
+                bm[k] = a;
+            }
+            float tmax = bm[0];
+#pragma unroll
+            for (int k = 1; k < T / 32; ++k) tmax = fmaxf(tmax, bm[k]);
+            const float m_new = fmaxf(m_run, tmax);
+            const bool rescale = (j > 0) && (m_new > m_run);
+            const float alpha = rescale ? ex2_approx((m_run - m_new) * kq) : 1.f;
+
+            // PNQ: quantize exp(S - m_new) per 32-column block (E8M0 from the block maximum).
+            uint32_t pw[T / 8];
+            uint32_t sfw = 0;
+            float lsum = 0.f;
+#pragma unroll
+            for (int k = 0; k < T / 32; ++k) {
+                const float pmax = ex2_approx((bm[k] - m_new) * kq);
+                const int e = block_exponent_f32(__float_as_uint(pmax), uos);
+                const float ne = -static_cast<float>(e);
+                float bsum = 0.f;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    float f[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        f[i] = ex2_approx(fmaf(sv[32 * k + 8 * g + i] - m_new, kq, ne));
+                        bsum += f[i];
+                    }
+                    pw[4 * k + g] = pack_e2m1x8(f);
+                }
+                sfw |= static_cast<uint32_t>(e + 127) << (8 * k);
+                if (!pnq) lsum = fmaf(bsum, exp2_neg_int(-e), lsum);
+            }
+            // P buffer and O are free once the previous P*V finished.
+            if (j > 0) {
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_o_done, (j - 1) & 1, abort_flag, p.status,
+                                                                kTimeoutCode, kTimeoutNs))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+            }
+            if (__any_sync(0xffffffffu, rescale)) {
+                const uint32_t obase = tbase + lane_base + C::kColO;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32_sync(obase + 32 * c, r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    tmem_st32(obase + 32 * c, r);
+                }
+                {
+                    uint32_t r[16];
+                    tmem_ld16_sync(obase + D, r);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    tmem_st16(obase + D, r);
+                }
+                tmem_st_wait();
+            }
+            // P row -> shared memory in the swizzled K-major layout the MMA reads.
+            {
+                uint8_t* prow = sP + row * (T / 2);
+#pragma unroll
+                for (int c = 0; c < T / 32; ++c) {
+                    const int phys = (T == 128) ? (c ^ ((row >> 1) & 3)) : (c ^ ((row >> 2) & 1));
+                    *reinterpret_cast<uint4*>(prow + 16 * phys) =
+                        make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+                }
+                reinterpret_cast<uint32_t*>(sPsf)[(row & 31) * 4 + (row >> 5)] = sfw;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            mbar_arrive(bar_p_full);
+            l_run = fmaf(l_run, alpha, lsum);
+            m_run = m_new;
+        }
+        // Epilogue: O / l for the valid rows.
+        if (ok && __all_sync(0xffffffffu, mbar_wait_bounded(bar_o_done, (nkv - 1) & 1, abort_flag, p.status,
+                                                             kTimeoutCode, kTimeoutNs))) {
+            tc_fence_after_sync();
+            const uint32_t obase = tbase + lane_base + C::kColO;
+            uint32_t lr[16];
+            tmem_ld16_sync(obase + D, lr);
+            const float l = pnq ? __uint_as_float(lr[0]) : l_run;
+            const float inv_l = 1.f / l;
+            const int qrow = qt * 128 + row;
+            float* out = p.O + (static_cast<size_t>(bh) * p.N + qrow) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32_sync(obase + 32 * c, r);
+                if (qrow < p.N) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4*>(out + 32 * c + i) =
+                            make_float4(__uint_as_float(r[i]) * inv_l, __uint_as_float(r[i + 1]) * inv_l,
+                                        __uint_as_float(r[i + 2]) * inv_l, __uint_as_float(r[i + 3]) * inv_l);
+                }
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after_sync();
+        tmem_dealloc(tbase, 512);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 3-D byte tensor [outer, rows, inner_bytes] with a (box_inner x box_rows x 1) box.
+bool encode_map(CUtensorMap* map, const void* base, uint64_t inner_bytes, uint64_t rows, uint64_t outer,
+                uint32_t box_inner, uint32_t box_rows) {
+    auto fn = get_encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[3] = {inner_bytes, rows, outer};
+    cuuint64_t strides[2] = {inner_bytes, inner_bytes * rows};
+    cuuint32_t box[3] = {box_inner, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle sw = (box_inner == 64) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, int T>
+cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
+    using C = Cfg<D, T>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int npad = (a.N + 31) / 32 * 32;
+    CUtensorMap tq, tk, tv;
+    if (!encode_map(&tq, a.q_codes, D / 2, a.N, a.BH, D / 2, 128) ||
+        !encode_map(&tk, a.k_codes, D / 2, a.N, a.BH, D / 2, T) ||
+        !encode_map(&tv, a.vt_codes, npad / 2, D, a.BH, T / 2, D))
+        return cudaErrorInvalidValue;
+    KParams kp{};
+    kp.q_sf = a.q_sf;
+    kp.k_sf = a.k_sf;
+    kp.v_sf = a.v_sf;
+    kp.O = a.O;
+    kp.status = a.status;
+    kp.N = a.N;
+    kp.ntq = (a.N + 127) / 128;
+    kp.nkv = (a.N + T - 1) / T;
+    kp.groups = (a.N + 127) / 128;
+    kp.pnq = a.pnq;
+    kp.uos = a.uos;
+    kp.kq = static_cast<float>(static_cast<double>(a.softmax_scale) * 1.4426950408889634);
+    dim3 grid(static_cast<unsigned>(a.BH * kp.ntq));
+    mxattn_fwd_kernel<D, T><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, kp);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
+    if (a.d == 128 && a.kv_tile == 128) return launch_impl<128, 128>(a, stream);
+    if (a.d == 128 && a.kv_tile == 64) return launch_impl<128, 64>(a, stream);
+    if (a.d == 64 && a.kv_tile == 128) return launch_impl<64, 128>(a, stream);
+    if (a.d == 64 && a.kv_tile == 64) return launch_impl<64, 64>(a, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace mxattn

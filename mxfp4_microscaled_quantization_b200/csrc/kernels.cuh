@@ -1,0 +1,50 @@
+// kernels.cuh -- host-side launchers shared by the C-ABI entry points.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace mxattn {
+
+// Row quantization of `ntensors` (1 or 2) bf16 tensors of shape [rows, cols].
+// regroup = 0: row-major scales; regroup = 1: rows are (bh, r < N), scales in
+// the 128-row regrouped order (padding rows zeroed).  Clears *status when
+// status != nullptr.
+cudaError_t launch_quantize_rows(const void* const* x, uint8_t* const* codes, uint8_t* const* scales, int ntensors,
+                                 int64_t rows, int cols, int uos, int regroup, int N, int groups, int64_t BH,
+                                 uint32_t* status, cudaStream_t stream);
+
+// V [BH, N, d] -> V^T codes [BH, d, Npad/2] and scales (row-major
+// [BH, d, Npad/32] when regroup = 0, regrouped per 128 tokens when 1).
+cudaError_t launch_quantize_vt(const void* v, int64_t BH, int N, int d, int uos, int regroup, int groups,
+                               uint8_t* codes_t, uint8_t* scales_t, cudaStream_t stream);
+
+// Row-major Q/K/V^T scales -> regrouped scales; clears *status.
+cudaError_t launch_regroup_sf(const uint8_t* q_scales, const uint8_t* k_scales, const uint8_t* vt_scales, int64_t BH,
+                              int N, int d, int groups, uint8_t* q_sf, uint8_t* k_sf, uint8_t* v_sf,
+                              uint32_t* status, cudaStream_t stream);
+
+struct AttnArgs {
+    const uint8_t* q_codes;  // [BH, N, d/2]
+    const uint8_t* k_codes;  // [BH, N, d/2]
+    const uint8_t* vt_codes; // [BH, d, Npad/2]
+    const uint8_t* q_sf;     // regrouped, [BH, G, 512]
+    const uint8_t* k_sf;
+    const uint8_t* v_sf;
+    float* O;                // [BH, N, d]
+    uint32_t* status;
+    int64_t BH;
+    int N;
+    int d;
+    int kv_tile;
+    int pnq;
+    int uos;
+    float softmax_scale;
+};
+
+// The fused attention kernel.  Returns cudaSuccess or the launch / encode error.
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream);
+
+}  // namespace mxattn

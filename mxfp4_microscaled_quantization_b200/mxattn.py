@@ -1,0 +1,239 @@
+"""ctypes binding of libmxattn.so (C ABI in include/mxattn.h).
+
+The functions carry the C names and only marshal arguments: torch tensors in,
+raw device pointers and sizes out, the current CUDA stream passed through.
+All compute happens in the library's CUDA kernels; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmxattn.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "mxattn.h")
+
+STATUS = {0: "MXATTN_OK", 1: "MXATTN_ERR_INVALID", 2: "MXATTN_ERR_UNSUPPORTED", 3: "MXATTN_ERR_CUDA",
+          4: "MXATTN_ERR_TIMEOUT"}
+RULES = {"ocp": 0, "uos": 1}
+
+
+class MxattnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmxattn.so (raises if it was not built: there is no CPU fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m mxfp4_microscaled_quantization_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i64, i32, u64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.mxattn_status_string.argtypes = [i32]
+        L.mxattn_status_string.restype = ctypes.c_char_p
+        L.mxattn_quantize.argtypes = [P, i64, i64, i32, P, P, P]
+        L.mxattn_quantize.restype = i32
+        L.mxattn_quantize_vt.argtypes = [P, i64, i64, i64, i32, P, P, P]
+        L.mxattn_quantize_vt.restype = i32
+        L.mxattn_workspace_size.argtypes = [i32, i32, i32, i32]
+        L.mxattn_workspace_size.restype = u64
+        L.mxattn_forward.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, ctypes.c_float, P, P, u64, P]
+        L.mxattn_forward.restype = i32
+        L.mxattn_prepare.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, u64, P]
+        L.mxattn_prepare.restype = i32
+        L.mxattn_attend.argtypes = [i32, i32, i32, i32, i32, i32, i32, ctypes.c_float, P, P, u64, P]
+        L.mxattn_attend.restype = i32
+        L.mxattn_forward_quantized.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
+                                               ctypes.c_float, P, P, u64, P]
+        L.mxattn_forward_quantized.restype = i32
+        L.mxattn_workspace_status.argtypes = [P, P]
+        L.mxattn_workspace_status.restype = i32
+        _lib = L
+    return _lib
+
+
+def declared_symbols() -> list[str]:
+    """Names of the entry points declared in include/mxattn.h."""
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"\b(mxattn_[a-z_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return lib().mxattn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise MxattnError(status, where)
+
+
+def _rule(rule) -> int:
+    return RULES[rule] if isinstance(rule, str) else int(rule)
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def mxattn_quantize(x: torch.Tensor, rule="uos", codes=None, scales=None, stream=None):
+    """bf16 [..., cols] -> (codes u8 [..., cols/2], scales u8 [..., cols/32])."""
+    cols = x.shape[-1]
+    rows = x.numel() // cols if cols else 0
+    if codes is None:
+        codes = torch.empty(x.shape[:-1] + (cols // 2,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1] + (cols // 32,), dtype=torch.uint8, device=x.device)
+    _check(lib().mxattn_quantize(_cuda(x, "x", torch.bfloat16), rows, cols, _rule(rule), _cuda(codes, "codes"),
+                                 _cuda(scales, "scales"), _stream(stream)), "mxattn_quantize")
+    return codes, scales
+
+
+def mxattn_quantize_vt(v: torch.Tensor, rule="uos", codes_t=None, scales_t=None, stream=None):
+    """V bf16 [..., N, d] -> V^T (codes u8 [..., d, Npad/2], scales u8 [..., d, Npad/32])."""
+    N, d = v.shape[-2:]
+    BH = v.numel() // (N * d)
+    npad = (N + 31) // 32 * 32
+    lead = tuple(v.shape[:-2])
+    if codes_t is None:
+        codes_t = torch.empty(lead + (d, npad // 2), dtype=torch.uint8, device=v.device)
+    if scales_t is None:
+        scales_t = torch.empty(lead + (d, npad // 32), dtype=torch.uint8, device=v.device)
+    _check(lib().mxattn_quantize_vt(_cuda(v, "v", torch.bfloat16), BH, N, d, _rule(rule), _cuda(codes_t, "codes_t"),
+                                    _cuda(scales_t, "scales_t"), _stream(stream)), "mxattn_quantize_vt")
+    return codes_t, scales_t
+
+
+def mxattn_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().mxattn_workspace_size(B, H, N, d))
+
+
+def workspace_layout(B: int, H: int, N: int, d: int) -> dict:
+    """Byte offsets of the workspace regions (as documented in include/mxattn.h)."""
+    a = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    BH, G, npad = B * H, (N + 127) // 128, (N + 31) // 32 * 32
+    off, out = 0, {}
+    for name, size in (("status", 256), ("q_codes", BH * N * d // 2), ("k_codes", BH * N * d // 2),
+                       ("vt_codes", BH * d * npad // 2), ("q_sf", BH * G * 512), ("k_sf", BH * G * 512),
+                       ("vt_sf", BH * G * 512)):
+        out[name] = (off, size)
+        off = a(off + size)
+    out["total"] = off
+    return out
+
+
+def new_workspace(B, H, N, d, device="cuda") -> torch.Tensor:
+    n = mxattn_workspace_size(B, H, N, d)
+    if n == 0:
+        raise MxattnError(1, "mxattn_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def mxattn_forward(q, k, v, kv_tile=128, pnq=True, rule="uos", softmax_scale=0.0, out=None, workspace=None,
+                   stream=None):
+    """Fused MXFP4 attention: q, k, v bf16 [B, H, N, d] -> O fp32 [B, H, N, d]."""
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(B, H, N, d, q.device)
+    _check(lib().mxattn_forward(_cuda(q, "q", torch.bfloat16), _cuda(k, "k", torch.bfloat16),
+                                _cuda(v, "v", torch.bfloat16), B, H, N, d, kv_tile, 1 if pnq else 0, _rule(rule),
+                                float(softmax_scale), _cuda(out, "out", torch.float32), _cuda(workspace, "workspace"),
+                                workspace.numel(), _stream(stream)), "mxattn_forward")
+    return out
+
+
+def mxattn_prepare(q, k, v, rule="uos", workspace=None, stream=None):
+    """Quantize q, k, v (bf16 [B, H, N, d]) into `workspace` (the first half of mxattn_forward)."""
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    if workspace is None:
+        workspace = new_workspace(B, H, N, d, q.device)
+    _check(lib().mxattn_prepare(_cuda(q, "q", torch.bfloat16), _cuda(k, "k", torch.bfloat16),
+                                _cuda(v, "v", torch.bfloat16), B, H, N, d, _rule(rule), _cuda(workspace, "workspace"),
+                                workspace.numel(), _stream(stream)), "mxattn_prepare")
+    return workspace
+
+
+def mxattn_attend(workspace, B, H, N, d, kv_tile=128, pnq=True, rule="uos", softmax_scale=0.0, out=None, stream=None):
+    """Attention on a workspace filled by mxattn_prepare (the second half of mxattn_forward)."""
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.float32, device=workspace.device)
+    _check(lib().mxattn_attend(B, H, N, d, kv_tile, 1 if pnq else 0, _rule(rule), float(softmax_scale),
+                               _cuda(out, "out", torch.float32), _cuda(workspace, "workspace"), workspace.numel(),
+                               _stream(stream)), "mxattn_attend")
+    return out
+
+
+def mxattn_forward_quantized(q_codes, q_scales, k_codes, k_scales, vt_codes, vt_scales, B, H, N, d, kv_tile=128,
+                             pnq=True, rule="uos", softmax_scale=0.0, out=None, workspace=None, stream=None):
+    """Attention on operands already quantized in the public layouts."""
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.float32, device=q_codes.device)
+    if workspace is None:
+        workspace = new_workspace(B, H, N, d, q_codes.device)
+    _check(lib().mxattn_forward_quantized(
+        _cuda(q_codes, "q_codes"), _cuda(q_scales, "q_scales"), _cuda(k_codes, "k_codes"),
+        _cuda(k_scales, "k_scales"), _cuda(vt_codes, "vt_codes"), _cuda(vt_scales, "vt_scales"),
+        B, H, N, d, kv_tile, 1 if pnq else 0, _rule(rule), float(softmax_scale), _cuda(out, "out", torch.float32),
+        _cuda(workspace, "workspace"), workspace.numel(), _stream(stream)), "mxattn_forward_quantized")
+    return out
+
+
+def mxattn_workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronize and return the status word of the last forward on `workspace` (0 = ok)."""
+    return int(lib().mxattn_workspace_status(_cuda(workspace, "workspace"), _stream(stream)))
+
+
+def mxattn_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def attention_from_host(q_host, k_host, v_host, kv_tile=128, pnq=True, rule="uos", softmax_scale=0.0,
+                        device_buffers=None, out_host=None, stream=None):
+    """End-to-end call with host tensors: copy q, k, v (pinned host bf16) to the
+    device, run mxattn_forward, copy O back into `out_host` (pinned fp32).
+    `device_buffers` = (q, k, v, out, workspace) device tensors to reuse."""
+    B, H, N, d = q_host.shape
+    if device_buffers is None:
+        dev = torch.device("cuda")
+        device_buffers = (torch.empty_like(q_host, device=dev), torch.empty_like(k_host, device=dev),
+                          torch.empty_like(v_host, device=dev),
+                          torch.empty((B, H, N, d), dtype=torch.float32, device=dev), new_workspace(B, H, N, d))
+    qd, kd, vd, od, ws = device_buffers
+    qd.copy_(q_host, non_blocking=True)
+    kd.copy_(k_host, non_blocking=True)
+    vd.copy_(v_host, non_blocking=True)
+    mxattn_forward(qd, kd, vd, kv_tile, pnq, rule, softmax_scale, od, ws, stream)
+    if out_host is None:
+        out_host = torch.empty((B, H, N, d), dtype=torch.float32, pin_memory=True)
+    out_host.copy_(od, non_blocking=True)
+    return out_host

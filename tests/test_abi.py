@@ -1,0 +1,87 @@
+"""The C-ABI library builds, loads and exports what include/mxattn.h declares;
+host-side argument checks (no GPU: every call here returns before any CUDA call)."""
+import ctypes
+import subprocess
+
+import pytest
+
+from mxfp4_microscaled_quantization_b200 import build as build_mod
+from mxfp4_microscaled_quantization_b200 import mxattn as mx
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_mod.build()
+    return mx.lib()
+
+
+def test_header_declares_the_boundary():
+    syms = mx.declared_symbols()
+    for name in ("mxattn_quantize", "mxattn_quantize_vt", "mxattn_workspace_size", "mxattn_forward",
+                 "mxattn_forward_quantized", "mxattn_workspace_status", "mxattn_status_string", "mxattn_prepare",
+                 "mxattn_attend"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in mx.declared_symbols():
+        assert hasattr(L, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", mx.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(mx.declared_symbols()) <= exported
+    # nothing but the C ABI is exported from the library's own code
+    assert not [s for s in exported if s.startswith("_ZN6mxattn")]
+
+
+def test_status_strings(L):
+    for s in range(5):
+        assert isinstance(mx.status_string(s), str) and mx.status_string(s)
+    assert mx.status_string(99) == "unknown status"
+
+
+def test_workspace_size_matches_documented_layout(L):
+    for shape in ((1, 1, 256, 64), (1, 8, 4096, 128), (1, 40, 32760, 128), (2, 3, 1, 64), (1, 1, 129, 128)):
+        assert mx.mxattn_workspace_size(*shape) == mx.workspace_layout(*shape)["total"]
+    assert mx.mxattn_workspace_size(1, 1, 256, 96) == 0
+    assert mx.mxattn_workspace_size(1, 1, 0, 64) == 0
+    assert mx.mxattn_workspace_size(0, 1, 16, 64) == 0
+
+
+def _p(x):
+    return ctypes.c_void_p(x)
+
+
+def test_quantize_rejects_bad_arguments_before_launching(L):
+    fake = _p(1 << 20)
+    assert L.mxattn_quantize(fake, 4, 48, 1, fake, fake, None) == 1        # cols % 32 != 0
+    assert L.mxattn_quantize(fake, -1, 64, 1, fake, fake, None) == 1       # negative rows
+    assert L.mxattn_quantize(fake, 4, 64, 7, fake, fake, None) == 1        # unknown rule
+    assert L.mxattn_quantize(None, 4, 64, 1, fake, fake, None) == 1        # null input
+    assert L.mxattn_quantize(_p((1 << 20) + 8), 4, 64, 1, fake, fake, None) == 1  # misaligned input
+    assert L.mxattn_quantize(None, 0, 64, 1, None, None, None) == 0        # empty is a no-op
+    assert L.mxattn_quantize_vt(fake, 1, 16, 96, 1, fake, fake, None) == 2  # d unsupported
+    assert L.mxattn_quantize_vt(fake, 1, 0, 64, 1, fake, fake, None) == 1   # N < 1
+
+
+def test_forward_rejects_bad_arguments_before_launching(L):
+    fake = _p(1 << 20)
+    ws_ok = mx.mxattn_workspace_size(1, 1, 256, 64)
+    args = lambda d=64, t=64, pnq=1, rule=1, N=256, ws=ws_ok, o=fake: (  # noqa: E731
+        fake, fake, fake, 1, 1, N, d, t, pnq, rule, ctypes.c_float(0.0), o, fake, ws, None)
+    assert L.mxattn_forward(*args(d=96)) == 2
+    assert L.mxattn_forward(*args(t=32)) == 2
+    assert L.mxattn_forward(*args(pnq=2)) == 1
+    assert L.mxattn_forward(*args(rule=3)) == 1
+    assert L.mxattn_forward(*args(N=0)) == 1
+    assert L.mxattn_forward(*args(ws=ws_ok - 1)) == 1
+    assert L.mxattn_forward(*args(o=None)) == 1
+    assert L.mxattn_forward(*args(N=(1 << 24) + 1, ws=1 << 40)) == 2
+    q = (fake,) * 6
+    assert L.mxattn_forward_quantized(*q, 1, 1, 256, 64, 96, 1, 1, ctypes.c_float(0), fake, fake, ws_ok, None) == 2
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(mx, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(mx, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        mx.lib()
