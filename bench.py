@@ -78,7 +78,7 @@ def profiled_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 200 ms during the timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms during the timed region."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -93,7 +93,7 @@ class ClockSampler:
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-i", str(self.gpu), "-lms", "200"], stdout=self.fh,
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=self.fh,
                                          stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -141,22 +141,29 @@ def oracle_sample(Q, K, V, w, rows, nthreads=0):
     return time.perf_counter() - t0
 
 
+def sized_oracle_rows(Q, K, V, w, budget_s, threads):
+    """Grow a seeded row sample until one oracle call takes about `budget_s` (or all rows)."""
+    n = 2 * threads
+    for _ in range(4):
+        rows = np.linspace(0, w.N - 1, n).astype(np.int64)
+        t = oracle_sample(Q, K, V, w, rows, threads)
+        if t >= 0.5 * budget_s or n >= w.N:
+            return rows, t
+        n = int(min(w.N, max(n + 1, n * budget_s / max(t, 1e-3))))
+    return rows, t
+
+
 def cpu_baseline(Q, K, V, w, budget_s=15.0):
     """Time the oracle as it stands on a bounded sample: query rows of head 0 sized to
     about `budget_s` of CPU work, converted to the same unit (4*N*d flops per row)."""
     import oracle
 
     threads = oracle.max_threads()
-    probe = np.arange(0, w.N, max(1, w.N // (2 * threads)))[: 2 * threads]
-    t = oracle_sample(Q, K, V, w, probe, threads)
-    per_row = t / len(probe)
-    n = int(min(w.N, max(len(probe), budget_s / max(per_row, 1e-9))))
-    rows = np.linspace(0, w.N - 1, n).astype(np.int64)
-    t = oracle_sample(Q, K, V, w, rows, threads)
-    flops = 4.0 * n * w.N * w.d
+    rows, t = sized_oracle_rows(Q, K, V, w, budget_s, threads)
+    flops = 4.0 * len(rows) * w.N * w.d
     return {"value": flops / t / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{n} query rows of head 0 of {w.name} (full K/V quantization of that head included), "
-                      f"{t:.1f} s on {threads} OpenMP threads"}
+            "sample": f"{len(rows)} evenly spaced query rows of head 0 of {w.name} (that head's K/V quantization "
+                      f"included), {t:.1f} s on {threads} OpenMP threads"}
 
 
 def run_reference(args, rank, world):
@@ -169,10 +176,9 @@ def run_reference(args, rank, world):
     Q, K, V = wl.make_qkv(w, seed=0)
     threads = oracle.max_threads()
     # size one step to a bounded sample so warmup + steps stay within a few minutes
-    probe = np.arange(threads) * (w.N // threads)
-    per_row = oracle_sample(Q, K, V, w, probe, threads) / len(probe)
-    step_budget_s = max(2.0, 120.0 / (args.warmup + args.steps))  # whole run within a few minutes
-    n = int(max(threads, min(w.N, step_budget_s / max(per_row, 1e-9))))
+    step_budget_s = max(2.0, 120.0 / (args.warmup + args.steps))
+    rows0, _ = sized_oracle_rows(Q, K, V, w, step_budget_s, threads)
+    n = len(rows0)
     times = []
     for i in range(args.warmup + args.steps):
         rng = np.random.default_rng(i)
@@ -221,6 +227,30 @@ def quantize_sweep_point(torch, mx, peaks, peak_kind, log2n=30, iters=10):
     return out
 
 
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of per-rank timings (the slowest rank counts); identity without a process group."""
+    import torch
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own batch (weak scaling: one independent problem per GPU)."""
+    return rank
+
+
+def selected_workload(args):
+    w = wl.WORKLOADS[args.workload]
+    if args.heads:
+        import dataclasses
+
+        w = dataclasses.replace(w, H=args.heads)
+    return w
+
+
 def run_gpu(args, rank, world, local_rank):
     import torch
 
@@ -234,13 +264,13 @@ def run_gpu(args, rank, world, local_rank):
         import torch.distributed as dist
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    w = WORKLOAD
+    w = selected_workload(args)
     peaks, peak_kind = load_peaks()
     B, H, N, d = w.B, w.H, w.N, w.d
 
-    Q, K, V = wl.make_qkv(w, seed=rank)
+    Q, K, V = wl.make_qkv(w, seed=rank_seed(rank))
     base = None
-    if rank == 0:
+    if rank == 0 and not args.quick:
         base = cpu_baseline(Q, K, V, w, budget_s=args.cpu_budget)
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)  # noqa: E731
     q, k, v = to_dev(Q), to_dev(K), to_dev(V)
@@ -279,19 +309,59 @@ def run_gpu(args, rank, world, local_rank):
     prep_ms = [e[0].elapsed_time(e[1]) for e in evs]
     if mx.mxattn_workspace_status(ws) != 0:
         raise RuntimeError("attention kernel reported a timeout")
-    t = torch.tensor([total_ms, sum(attn_ms) / len(attn_ms)], dtype=torch.float64, device="cuda")
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, attn_avg_ms = float(t[0]), float(t[1])
+    total_ms, attn_avg_ms = max_over_ranks([total_ms, sum(attn_ms) / len(attn_ms)], dist, "cuda")
     ms_per_step = total_ms / args.steps
     value = world * w.flops / (ms_per_step / 1e3) / 1e12
 
-    # end to end through the public API with host buffers (pinned), H2D + D2H inside the timed region
+    e2e_ms = None
+    if not args.quick:
+        e2e_ms = measure_e2e(torch, mx, Q, K, V, w, (q, k, v, out, ws), stream, args, dist)
+
+    quant = None
+    if rank == 0 and not args.quick and not args.no_quantize_sweep:
+        quant = quantize_sweep_point(torch, mx, peaks, peak_kind)
+
+    if rank == 0:
+        attn_tflops = w.flops / (attn_avg_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
+        clocks = clk.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "mxfp4 (e2m1 x e8m0, fp32 accumulate)", "data": "synthetic",
+            "config": {**config_dict(w), "parallelism": f"{world} independent replicas (one batch per rank)"},
+            "pct_of_fp4_peak": 100.0 * value / world / peak,
+            "roofline": {"bound": "tensor", "kernel": f"mxattn_fwd_kernel<{w.d},{w.kv_tile}>", "achieved": attn_tflops,
+                         "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                         "traffic": profiled_traffic() if w == WORKLOAD else None,
+                         "peak_source": f"{peak_kind} bf16 sustained {peaks['bf16_tflops_sustained']} TFLOP/s x "
+                                        f"{FP4_PER_BF16:g} (nominal dense fp4:bf16)",
+                         "attn_ms": attn_avg_ms, "prepare_ms": sum(prep_ms) / len(prep_ms),
+                         "frac_of_9pf_spec": attn_tflops / 9000.0},
+            "cpu_baseline": base,
+            "e2e": None if e2e_ms is None else {
+                "value": world * w.flops / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": 3 * B * H * N * d * 2, "d2h_bytes_per_step": B * H * N * d * 4,
+                "ms_per_step": e2e_ms, "api": "attention_from_host -> mxattn_forward"},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks,
+            "quantize_sweep": quant,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def measure_e2e(torch, mx, Q, K, V, w, bufs, stream, args, dist):
+    """Same metric end to end through the public API with pinned host buffers:
+    H2D of Q/K/V and D2H of O inside the timed region."""
+    B, H, N, d = w.B, w.H, w.N, w.d
     q_h = torch.from_numpy(Q.view(np.int16)).view(torch.bfloat16).pin_memory()
     k_h = torch.from_numpy(K.view(np.int16)).view(torch.bfloat16).pin_memory()
     v_h = torch.from_numpy(V.view(np.int16)).view(torch.bfloat16).pin_memory()
     o_h = torch.empty((B, H, N, d), dtype=torch.float32).pin_memory()
-    bufs = (q, k, v, out, ws)
     for _ in range(2):
         mx.attention_from_host(q_h, k_h, v_h, w.kv_tile, True, "uos", 0.0, bufs, o_h)
     torch.cuda.synchronize()
@@ -304,55 +374,22 @@ def run_gpu(args, rank, world, local_rank):
         mx.attention_from_host(q_h, k_h, v_h, w.kv_tile, True, "uos", 0.0, bufs, o_h)
     ee1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([ee0.elapsed_time(ee1) / e2e_steps], dtype=torch.float64, device="cuda")
-    if dist is not None:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te[0])
-
-    quant = None
-    if rank == 0 and not args.no_quantize_sweep:
-        quant = quantize_sweep_point(torch, mx, peaks, peak_kind)
-
-    if rank == 0:
-        attn_tflops = w.flops / (attn_avg_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
-        clocks = clk.summary()
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "mxfp4 (e2m1 x e8m0, fp32 accumulate)", "data": "synthetic",
-            "config": {**config_dict(), "parallelism": f"{world} independent replicas (one batch per rank)"},
-            "pct_of_fp4_peak": 100.0 * value / world / peak,
-            "roofline": {"bound": "tensor", "kernel": "mxattn_fwd_kernel<128,128>", "achieved": attn_tflops,
-                         "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
-                         "traffic": profiled_traffic(),
-                         "peak_source": f"{peak_kind} bf16 sustained {peaks['bf16_tflops_sustained']} TFLOP/s x "
-                                        f"{FP4_PER_BF16:g} (nominal dense fp4:bf16)",
-                         "attn_ms": attn_avg_ms, "prepare_ms": sum(prep_ms) / len(prep_ms),
-                         "frac_of_9pf_spec": attn_tflops / 9000.0},
-            "cpu_baseline": base,
-            "e2e": {"value": world * w.flops / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
-                    "h2d_bytes_per_step": 3 * B * H * N * d * 2, "d2h_bytes_per_step": B * H * N * d * 4,
-                    "ms_per_step": e2e_ms, "api": "attention_from_host -> mxattn_forward"},
-            "gpu_launches": 3 * args.steps,
-            "clocks": clocks,
-            "quantize_sweep": quant,
-        }
-        print(json.dumps(line), flush=True)
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
-    return 0
+    return max_over_ranks([ee0.elapsed_time(ee1) / e2e_steps], dist, "cuda")[0]
 
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-quantize-sweep", action="store_true")
+    ap.add_argument("--workload", choices=sorted(wl.WORKLOADS), default="video_dit",
+                    help="workload to time (default: the video-DiT configuration the metric is quoted on)")
+    ap.add_argument("--heads", type=int, default=0, help="override H (smaller cases for profiling)")
+    ap.add_argument("--quick", action="store_true",
+                    help="timed steps only: no CPU baseline, no end-to-end leg, no quantize sweep")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))

@@ -7,17 +7,19 @@
 // is built from the same quantized values that weight V (PNQ).
 //
 // One CTA owns 128 query rows of one (batch, head) and walks all key tiles in
-// ascending order.  Roles (192 threads):
-//   warp 4 (one lane)  TMA producer: Q tile + scales once, then K and V^T
-//                      tiles (+ scales) into a kStages-deep ring.
-//   warp 5 (one lane)  MMA issuer: tcgen05.cp of E8M0 scales into TMEM and
-//                      tcgen05.mma kind::mxf4 block_scale for S = Q K^T
-//                      (double-buffered in TMEM) and O += P V.
-//   warps 0-3          softmax, one thread per query row (= TMEM lane):
-//                      running max, exp2 on the MUFU, per-32-column block
-//                      exponent (UOS/OCP), E2M1 packing of P into shared
+// ascending order.  Roles (320 threads):
+//   warps 0-7          softmax, two threads per query row (= TMEM lane), each
+//                      owning half of every S tile's columns: partial row max
+//                      (exchanged through shared memory and an mbarrier),
+//                      exp2 on the MUFU with packed f32x2 FMAs, per-32-column
+//                      block exponent (UOS/OCP), E2M1 packing of P into shared
 //                      memory, O rescale in TMEM when the max moved, and the
 //                      final O / l.
+//   warp 8 (one lane)  TMA producer: Q tile + scales once, then K and V^T
+//                      tiles (+ scales) into a kStages-deep ring.
+//   warp 9 (one lane)  MMA issuer: tcgen05.cp of E8M0 scales into TMEM and
+//                      tcgen05.mma kind::mxf4 block_scale for S = Q K^T
+//                      (double-buffered in TMEM) and O += P V.
 // The row sum under PNQ is produced by the tensor core itself: V^T gets one
 // extra row of ones (E2M1 1.0, scale 2^0) so O's column d accumulates
 // sum_j q_j -- exactly the quantized values that multiply V -- and is
@@ -47,7 +49,14 @@ constexpr uint32_t kTimeoutCode = 4u;           // MXATTN_ERR_TIMEOUT
 template <int D, int T>
 struct Cfg {
     static constexpr int kStages = 4;
-    static constexpr int kThreads = 192;
+    static constexpr int kSplit = 2;                       // softmax threads per query row
+    static constexpr int kSoftThreads = 128 * kSplit;      // softmax warps 0 .. 4*kSplit-1
+    static constexpr int kProducerWarp = 4 * kSplit;
+    static constexpr int kMmaWarp = 4 * kSplit + 1;
+    static constexpr int kThreads = kSoftThreads + 64;
+    static constexpr int kCols = T / kSplit;               // S columns per softmax thread
+    static constexpr int kBlk = kCols / 32;                // P blocks per softmax thread
+    static_assert(kBlk >= 1, "each softmax thread owns at least one 32-column block");
     static constexpr int kQBytes = 128 * D / 2;
     static constexpr int kKBytes = T * D / 2;
     static constexpr int kVRows = D + 16;  // V^T rows + a row of ones + 15 zero rows
@@ -71,9 +80,11 @@ struct Cfg {
     static constexpr int kOffVsf = kOffKsf + kStages * kSfBytes;
     static constexpr int kOffPsf = kOffVsf + kStages * kSfBytes;
     static constexpr int kOffVsfConst = kOffPsf + kSfBytes;
-    static constexpr int kOffBar = kOffVsfConst + kSfBytes;
-    // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_empty[2], p_full, o_done, drain
-    static constexpr int kNumBars = 1 + 4 * kStages + 4 + 3;
+    static constexpr int kOffRed = kOffVsfConst + kSfBytes;     // float [2][kSplit][128] row-max exchange
+    static constexpr int kOffBar = kOffRed + 2 * kSplit * 128 * 4;
+    // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_empty[2], p_full, o_done, drain,
+    //           red[2], lsum
+    static constexpr int kNumBars = 1 + 4 * kStages + 4 + 3 + 3;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemUsed = kOffMisc + 16;
     // >= 116 KB keeps one CTA per SM, so the 512-column TMEM allocation never waits
@@ -101,18 +112,30 @@ struct KParams {
     int ntq;     // query tiles per head
     int nkv;     // key tiles per head
     int groups;  // 128-row scale groups per head
-    int pnq;
     int uos;
     float kq;    // softmax_scale * log2(e)
 };
+
+// Maximum of 32 values as a depth-4 tree of 3-input max instructions.
+__device__ __forceinline__ float block_max32(const float* v) {
+    float t[11];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) t[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+    t[10] = fmaxf(v[30], v[31]);
+    const float u0 = fmax3(t[0], t[1], t[2]);
+    const float u1 = fmax3(t[3], t[4], t[5]);
+    const float u2 = fmax3(t[6], t[7], t[8]);
+    const float u3 = fmaxf(t[9], t[10]);
+    return fmax3(u0, u1, fmaxf(u2, u3));
+}
 
 __device__ __forceinline__ uint64_t sf_desc(const void* p) {
     // 32 rows x 16 bytes, rows contiguous: core matrices of 8 rows 128 bytes apart
     return smem_desc(smem_u32(p), 0, 128, kLayoutNone);
 }
 
-template <int D, int T>
-__global__ void __launch_bounds__(192, 1)
+template <int D, int T, bool PNQ>
+__global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
     mxattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const KParams p) {
     using C = Cfg<D, T>;
@@ -140,6 +163,9 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* bar_p_full = bar_s_empty + 2;
     uint64_t* bar_o_done = bar_p_full + 1;
     uint64_t* bar_drain = bar_o_done + 1;
+    uint64_t* bar_red = bar_drain + 1;  // [2]
+    uint64_t* bar_lsum = bar_red + 2;
+    float* red = reinterpret_cast<float*>(smem + C::kOffRed);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -160,9 +186,11 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_s_full + b, 1);
-            mbar_init(bar_s_empty + b, 128);
+            mbar_init(bar_s_empty + b, C::kSoftThreads);
+            mbar_init(bar_red + b, C::kSoftThreads);
         }
-        mbar_init(bar_p_full, 128);
+        mbar_init(bar_lsum, C::kSoftThreads);
+        mbar_init(bar_p_full, C::kSoftThreads);
         mbar_init(bar_o_done, 1);
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
@@ -178,7 +206,7 @@ __global__ void __launch_bounds__(192, 1)
     // Scale factors of V^T rows 128..255 (only used when D = 128): all 2^0.
     for (int idx = tid; idx < 128; idx += C::kThreads) reinterpret_cast<uint32_t*>(sVsfConst)[idx] = 0x7F7F7F7Fu;
     fence_proxy_async_smem();
-    if (warp == 5) {
+    if (warp == C::kMmaWarp) {
         tmem_alloc(tmem_holder, 512);
         tmem_relinquish();
     }
@@ -187,7 +215,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after_sync();
     const uint32_t tbase = *tmem_holder;
 
-    if (warp == 4) {
+    if (warp == C::kProducerWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int k_issued = 0, v_issued = 0;
@@ -226,7 +254,7 @@ __global__ void __launch_bounds__(192, 1)
                     mbar_wait_bounded(bar_v_full + j % S, (j / S) & 1, no_abort, p.status, kTimeoutCode, kTimeoutNs);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == C::kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t t_s[2] = {tbase + C::kColS0, tbase + C::kColS1};
@@ -288,15 +316,19 @@ __global__ void __launch_bounds__(192, 1)
             mbar_wait_bounded(bar_drain, 0, &dummy, p.status, kTimeoutCode, kTimeoutNs);
         }
     } else {
-        // ------------------------------------------------------------ softmax (thread = query row)
-        const int row = tid;  // 0..127 == TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        // ------------------------------------------------------------ softmax
+        // kSplit threads per query row (= TMEM lane): thread `part` owns S columns
+        // [part*kCols, (part+1)*kCols) of every tile, i.e. kBlk 32-column P blocks.
+        constexpr int kCols = C::kCols;
+        constexpr int kBlk = C::kBlk;
+        const int row = tid & 127;
+        const int part = tid >> 7;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const float kq = p.kq;
         const int uos = p.uos;
-        const int pnq = p.pnq;
         const int valid_last = p.N - (nkv - 1) * T;
         float m_run = -INFINITY;
-        float l_run = 0.f;
+        float l_run = 0.f;  // PNQ off: this thread's share of the row sum
         bool ok = true;
         for (int j = 0; j < nkv; ++j) {
             const int b = j & 1;
@@ -306,60 +338,80 @@ __global__ void __launch_bounds__(192, 1)
                 break;
             }
             tc_fence_after_sync();
-            float sv[T];
+            float sv[kCols];
+            {
+                const uint32_t taddr = tbase + lane_base + (b ? C::kColS1 : C::kColS0) + part * kCols;
+                if constexpr (kCols == 64) {
+                    uint32_t r[64];
+                    tmem_ld64_sync(taddr, r);
 #pragma unroll
-            for (int c = 0; c < T / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32_sync(tbase + lane_base + (b ? C::kColS1 : C::kColS0) + 32 * c, r);
+                    for (int i = 0; i < 64; ++i) sv[i] = __uint_as_float(r[i]);
+                } else {
+                    uint32_t r[32];
+                    tmem_ld32_sync(taddr, r);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) sv[32 * c + i] = __uint_as_float(r[i]);
+                    for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(r[i]);
+                }
             }
             tc_fence_before_sync();
             mbar_arrive(bar_s_empty + b);
             if (j == nkv - 1 && valid_last < T) {
 #pragma unroll
-                for (int i = 0; i < T; ++i)
-                    if (i >= valid_last) sv[i] = -INFINITY;
+                for (int i = 0; i < kCols; ++i)
+                    if (part * kCols + i >= valid_last) sv[i] = -INFINITY;
             }
-            float bm[T / 32];
+            float bm[kBlk];
 #pragma unroll
-            for (int k = 0; k < T / 32; ++k) {
-                float a = sv[32 * k];
+            for (int k = 0; k < kBlk; ++k) bm[k] = block_max32(sv + 32 * k);
+            float lmax = bm[0];
 #pragma unroll
-                for (int i = 1; i < 32; ++i) a = fmaxf(a, sv[32 * k + i]);
-                bm[k] = a;
+            for (int k = 1; k < kBlk; ++k) lmax = fmaxf(lmax, bm[k]);
+            // exchange the partial maxima of the row's kSplit threads
+            red[(b * C::kSplit + part) * 128 + row] = lmax;
+            mbar_arrive(bar_red + b);
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_red + b, (j >> 1) & 1, abort_flag, p.status,
+                                                            kTimeoutCode, kTimeoutNs))) {
+                ok = false;
+                break;
             }
-            float tmax = bm[0];
+            float tmax = red[(b * C::kSplit) * 128 + row];
 #pragma unroll
-            for (int k = 1; k < T / 32; ++k) tmax = fmaxf(tmax, bm[k]);
+            for (int q = 1; q < C::kSplit; ++q) tmax = fmaxf(tmax, red[(b * C::kSplit + q) * 128 + row]);
             const float m_new = fmaxf(m_run, tmax);
             const bool rescale = (j > 0) && (m_new > m_run);
             const float alpha = rescale ? ex2_approx((m_run - m_new) * kq) : 1.f;
 
-            // PNQ: quantize exp(S - m_new) per 32-column block (E8M0 from the block maximum).
-            uint32_t pw[T / 8];
+            // PNQ: quantize exp(S - m_new) per 32-column block.  pmax = 2^((bm - m) * kq)
+            // gives the block exponent e; each element is then 2^(s*kq - (m*kq + e)).
+            uint32_t pw[kCols / 8];
             uint32_t sfw = 0;
             float lsum = 0.f;
 #pragma unroll
-            for (int k = 0; k < T / 32; ++k) {
+            for (int k = 0; k < kBlk; ++k) {
                 const float pmax = ex2_approx((bm[k] - m_new) * kq);
                 const int e = block_exponent_f32(__float_as_uint(pmax), uos);
-                const float ne = -static_cast<float>(e);
+                const float nbias = -fmaf(m_new, kq, static_cast<float>(e));
                 float bsum = 0.f;
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
                     float f[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        f[i] = ex2_approx(fmaf(sv[32 * k + 8 * g + i] - m_new, kq, ne));
-                        bsum += f[i];
+                    for (int i = 0; i < 8; i += 2) {
+                        float w0, w1;
+                        ffma2_bcast(w0, w1, sv[32 * k + 8 * g + i], sv[32 * k + 8 * g + i + 1], kq, nbias);
+                        f[i] = ex2_approx(w0);
+                        f[i + 1] = ex2_approx(w1);
+                    }
+                    if constexpr (!PNQ) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) bsum += f[i];
                     }
                     pw[4 * k + g] = pack_e2m1x8(f);
                 }
                 sfw |= static_cast<uint32_t>(e + 127) << (8 * k);
-                if (!pnq) lsum = fmaf(bsum, exp2_neg_int(-e), lsum);
+                if constexpr (!PNQ) lsum = fmaf(bsum, exp2_neg_int(-e), lsum);
             }
-            // P buffer and O are free once the previous P*V finished.
+            // The P buffer and O are free once the previous P*V finished.
             if (j > 0) {
                 if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_o_done, (j - 1) & 1, abort_flag, p.status,
                                                                 kTimeoutCode, kTimeoutNs))) {
@@ -369,62 +421,84 @@ __global__ void __launch_bounds__(192, 1)
                 tc_fence_after_sync();
             }
             if (__any_sync(0xffffffffu, rescale)) {
-                const uint32_t obase = tbase + lane_base + C::kColO;
+                // this thread's share of O's columns (part 0 also owns the row-sum columns under PNQ)
+                constexpr int kOCols = D / C::kSplit;
+                const uint32_t obase = tbase + lane_base + C::kColO + part * kOCols;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < kOCols / 32; ++c) {
                     uint32_t r[32];
                     tmem_ld32_sync(obase + 32 * c, r);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
                     tmem_st32(obase + 32 * c, r);
                 }
-                {
+                if (PNQ && part == 0) {
                     uint32_t r[16];
-                    tmem_ld16_sync(obase + D, r);
+                    tmem_ld16_sync(tbase + lane_base + C::kColO + D, r);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st16(obase + D, r);
+                    tmem_st16(tbase + lane_base + C::kColO + D, r);
                 }
                 tmem_st_wait();
             }
-            // P row -> shared memory in the swizzled K-major layout the MMA reads.
+            // P row share -> shared memory in the swizzled K-major layout the MMA reads.
             {
                 uint8_t* prow = sP + row * (T / 2);
 #pragma unroll
-                for (int c = 0; c < T / 32; ++c) {
+                for (int k = 0; k < kBlk; ++k) {
+                    const int c = part * kBlk + k;  // 16-byte chunk = one 32-column block
                     const int phys = (T == 128) ? (c ^ ((row >> 1) & 3)) : (c ^ ((row >> 2) & 1));
                     *reinterpret_cast<uint4*>(prow + 16 * phys) =
-                        make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+                        make_uint4(pw[4 * k], pw[4 * k + 1], pw[4 * k + 2], pw[4 * k + 3]);
                 }
-                reinterpret_cast<uint32_t*>(sPsf)[(row & 31) * 4 + (row >> 5)] = sfw;
+                uint8_t* sfp = sPsf + (row & 31) * 16 + (row >> 5) * 4 + part * kBlk;
+                if constexpr (kBlk == 2)
+                    *reinterpret_cast<uint16_t*>(sfp) = static_cast<uint16_t>(sfw);
+                else if constexpr (kBlk == 1)
+                    *sfp = static_cast<uint8_t>(sfw);
+                else
+                    *reinterpret_cast<uint32_t*>(sfp) = sfw;
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
             mbar_arrive(bar_p_full);
-            l_run = fmaf(l_run, alpha, lsum);
+            if constexpr (!PNQ) l_run = fmaf(l_run, alpha, lsum);
             m_run = m_new;
         }
         // Epilogue: O / l for the valid rows.
         if (ok && __all_sync(0xffffffffu, mbar_wait_bounded(bar_o_done, (nkv - 1) & 1, abort_flag, p.status,
                                                              kTimeoutCode, kTimeoutNs))) {
             tc_fence_after_sync();
-            const uint32_t obase = tbase + lane_base + C::kColO;
-            uint32_t lr[16];
-            tmem_ld16_sync(obase + D, lr);
-            const float l = pnq ? __uint_as_float(lr[0]) : l_run;
-            const float inv_l = 1.f / l;
-            const int qrow = qt * 128 + row;
-            float* out = p.O + (static_cast<size_t>(bh) * p.N + qrow) * D;
+            float l;
+            bool have_l = true;
+            if constexpr (PNQ) {
+                l = __uint_as_float(tmem_ld1_sync(tbase + lane_base + C::kColO + D));
+            } else {
+                red[part * 128 + row] = l_run;  // the exchange buffers are idle after the loop
+                mbar_arrive(bar_lsum);
+                have_l = __all_sync(0xffffffffu, mbar_wait_bounded(bar_lsum, 0, abort_flag, p.status,
+                                                                   kTimeoutCode, kTimeoutNs));
+                l = 0.f;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32_sync(obase + 32 * c, r);
-                if (qrow < p.N) {
+                for (int q = 0; q < C::kSplit; ++q) l += red[q * 128 + row];
+            }
+            if (have_l) {
+                const float inv_l = 1.f / l;
+                const int qrow = qt * 128 + row;
+                constexpr int kOCols = D / C::kSplit;
+                float* out = p.O + (static_cast<size_t>(bh) * p.N + qrow) * D + part * kOCols;
+                const uint32_t obase = tbase + lane_base + C::kColO + part * kOCols;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<float4*>(out + 32 * c + i) =
-                            make_float4(__uint_as_float(r[i]) * inv_l, __uint_as_float(r[i + 1]) * inv_l,
-                                        __uint_as_float(r[i + 2]) * inv_l, __uint_as_float(r[i + 3]) * inv_l);
+                for (int c = 0; c < kOCols / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32_sync(obase + 32 * c, r);
+                    if (qrow < p.N) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4*>(out + 32 * c + i) =
+                                make_float4(__uint_as_float(r[i]) * inv_l, __uint_as_float(r[i + 1]) * inv_l,
+                                            __uint_as_float(r[i + 2]) * inv_l, __uint_as_float(r[i + 3]) * inv_l);
+                    }
                 }
             }
         }
@@ -432,7 +506,7 @@ __global__ void __launch_bounds__(192, 1)
 
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == C::kMmaWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tbase, 512);
     }
@@ -466,13 +540,13 @@ bool encode_map(CUtensorMap* map, const void* base, uint64_t inner_bytes, uint64
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int T>
+template <int D, int T, bool PNQ>
 cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
     using C = Cfg<D, T>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, T, PNQ>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -492,21 +566,25 @@ cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
     kp.ntq = (a.N + 127) / 128;
     kp.nkv = (a.N + T - 1) / T;
     kp.groups = (a.N + 127) / 128;
-    kp.pnq = a.pnq;
     kp.uos = a.uos;
     kp.kq = static_cast<float>(static_cast<double>(a.softmax_scale) * 1.4426950408889634);
     dim3 grid(static_cast<unsigned>(a.BH * kp.ntq));
-    mxattn_fwd_kernel<D, T><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, kp);
+    mxattn_fwd_kernel<D, T, PNQ><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, kp);
     return cudaGetLastError();
 }
 
 }  // namespace
 
+template <int D, int T>
+cudaError_t launch_pnq(const AttnArgs& a, cudaStream_t stream) {
+    return a.pnq ? launch_impl<D, T, true>(a, stream) : launch_impl<D, T, false>(a, stream);
+}
+
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {
-    if (a.d == 128 && a.kv_tile == 128) return launch_impl<128, 128>(a, stream);
-    if (a.d == 128 && a.kv_tile == 64) return launch_impl<128, 64>(a, stream);
-    if (a.d == 64 && a.kv_tile == 128) return launch_impl<64, 128>(a, stream);
-    if (a.d == 64 && a.kv_tile == 64) return launch_impl<64, 64>(a, stream);
+    if (a.d == 128 && a.kv_tile == 128) return launch_pnq<128, 128>(a, stream);
+    if (a.d == 128 && a.kv_tile == 64) return launch_pnq<128, 64>(a, stream);
+    if (a.d == 64 && a.kv_tile == 128) return launch_pnq<64, 128>(a, stream);
+    if (a.d == 64 && a.kv_tile == 64) return launch_pnq<64, 64>(a, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -189,6 +189,44 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+
+__device__ __forceinline__ void tmem_ld64_sync(uint32_t taddr, uint32_t (&v)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : MXATTN_R8(0), MXATTN_R8(8), MXATTN_R8(16), MXATTN_R8(24), MXATTN_R8(32), MXATTN_R8(40),
+          MXATTN_R8(48), MXATTN_R8(56)
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&v)[64]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, "
+        "%33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, "
+        "%49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};" ::"r"(taddr),
+        MXATTN_W8(0), MXATTN_W8(8), MXATTN_W8(16), MXATTN_W8(24), MXATTN_W8(32), MXATTN_W8(40), MXATTN_W8(48),
+        MXATTN_W8(56)
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t tmem_ld1_sync(uint32_t taddr) {
+    uint32_t v;
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(v)
+        : "r"(taddr)
+        : "memory");
+    return v;
+}
+
 #undef MXATTN_R8
 #undef MXATTN_W8
 
@@ -219,6 +257,26 @@ __host__ __device__ constexpr uint32_t mxf4_idesc(uint32_t n, uint32_t sfa_id, u
            | (1u << 23)               // scale format E8M0
            | ((128u >> 4) << 24)      // M / 16
            | ((sfa_id & 3u) << 29);   // A scale-factor byte id
+}
+
+
+// max(a, b, c) in one instruction (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// (o0, o1) = (x0, x1) * k + (c, c) as one packed f32x2 FMA.
+__device__ __forceinline__ void ffma2_bcast(float& o0, float& o1, float x0, float x1, float k, float c) {
+    asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 b, {%4, %4};\n\t"
+        "mov.b64 c, {%5, %5};\n\t"
+        "fma.rn.f32x2 d, a, b, c;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(o0), "=f"(o1)
+        : "f"(x0), "f"(x1), "f"(k), "f"(c));
 }
 
 // ------------------------------------------------------------------ E2M1 / E8M0 helpers
