@@ -6,20 +6,23 @@
 // MXFP4 (scale rule UOS, Qmax = 7.25, or OCP) before the row sum, so the sum
 // is built from the same quantized values that weight V (PNQ).
 //
-// One CTA owns 128 query rows of one (batch, head) and walks all key tiles in
-// ascending order.  Roles (320 threads):
-//   warps 0-7          softmax, two threads per query row (= TMEM lane), each
-//                      owning half of every S tile's columns: partial row max
-//                      (exchanged through shared memory and an mbarrier),
-//                      exp2 on the MUFU with packed f32x2 FMAs, per-32-column
-//                      block exponent (UOS/OCP), E2M1 packing of P into shared
-//                      memory, O rescale in TMEM when the max moved, and the
-//                      final O / l.
-//   warp 8 (one lane)  TMA producer: Q tile + scales once, then K and V^T
-//                      tiles (+ scales) into a kStages-deep ring.
+// One CTA owns two 128-row query tiles (A and B) of one (batch, head) and
+// walks all key tiles in ascending order; both tiles share every K / V^T tile
+// and one TMEM buffer for S, and their softmax warpgroups run a half-step
+// apart (ping-pong), so one tile's serial phases (TMEM load, waits, O
+// rescale, P hand-off) overlap the other tile's exponentials.  Roles (320
+// threads):
+//   warps 0-3 / 4-7    softmax for tile A / B, one thread per query row (=
+//                      TMEM lane): running max, exp2 on the MUFU with packed
+//                      f32x2 FMAs, per-32-column block exponent (UOS/OCP),
+//                      E2M1 packing of P into shared memory, O rescale in TMEM
+//                      when the max moved, and the final O / l.
+//   warp 8 (one lane)  TMA producer: both Q tiles + scales once, then K and
+//                      V^T tiles (+ scales) into a kStages-deep ring.
 //   warp 9 (one lane)  MMA issuer: tcgen05.cp of E8M0 scales into TMEM and
-//                      tcgen05.mma kind::mxf4 block_scale for S = Q K^T
-//                      (double-buffered in TMEM) and O += P V.
+//                      tcgen05.mma kind::mxf4 block_scale, in the order
+//                      S_A(j), S_B(j), S_A(j+1) ... interleaved with
+//                      O_A += P_A V(j), O_B += P_B V(j).
 // The row sum under PNQ is produced by the tensor core itself: V^T gets one
 // extra row of ones (E2M1 1.0, scale 2^0) so O's column d accumulates
 // sum_j q_j -- exactly the quantized values that multiply V -- and is
@@ -49,14 +52,12 @@ constexpr uint32_t kTimeoutCode = 4u;           // MXATTN_ERR_TIMEOUT
 template <int D, int T>
 struct Cfg {
     static constexpr int kStages = 4;
-    static constexpr int kSplit = 2;                       // softmax threads per query row
-    static constexpr int kSoftThreads = 128 * kSplit;      // softmax warps 0 .. 4*kSplit-1
-    static constexpr int kProducerWarp = 4 * kSplit;
-    static constexpr int kMmaWarp = 4 * kSplit + 1;
+    static constexpr int kTiles = 2;                  // query tiles per CTA
+    static constexpr int kRows = 128 * kTiles;        // query rows per CTA
+    static constexpr int kSoftThreads = 128 * kTiles;
+    static constexpr int kProducerWarp = 4 * kTiles;
+    static constexpr int kMmaWarp = 4 * kTiles + 1;
     static constexpr int kThreads = kSoftThreads + 64;
-    static constexpr int kCols = T / kSplit;               // S columns per softmax thread
-    static constexpr int kBlk = kCols / 32;                // P blocks per softmax thread
-    static_assert(kBlk >= 1, "each softmax thread owns at least one 32-column block");
     static constexpr int kQBytes = 128 * D / 2;
     static constexpr int kKBytes = T * D / 2;
     static constexpr int kVRows = D + 16;  // V^T rows + a row of ones + 15 zero rows
@@ -64,6 +65,7 @@ struct Cfg {
     static constexpr int kVStride = ((kVRows * T / 2) + 1023) / 1024 * 1024;
     static constexpr int kPBytes = 128 * T / 2;
     static constexpr int kSfBytes = 512;
+    static constexpr int kOCols = D + 16;
 
     static constexpr uint32_t kQKLayout = (D == 128) ? kLayoutSw64 : kLayoutSw32;
     static constexpr uint32_t kQKSbo = 8 * D / 2;
@@ -71,35 +73,34 @@ struct Cfg {
     static constexpr uint32_t kPVSbo = 8 * T / 2;
 
     // shared memory (offsets from a 1024-aligned base)
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kQBytes;
-    static constexpr int kOffV = kOffK + kStages * kKBytes;
-    static constexpr int kOffP = kOffV + kStages * kVStride;
-    static constexpr int kOffQsf = kOffP + kPBytes;
-    static constexpr int kOffKsf = kOffQsf + kSfBytes;
-    static constexpr int kOffVsf = kOffKsf + kStages * kSfBytes;
-    static constexpr int kOffPsf = kOffVsf + kStages * kSfBytes;
-    static constexpr int kOffVsfConst = kOffPsf + kSfBytes;
-    static constexpr int kOffRed = kOffVsfConst + kSfBytes;     // float [2][kSplit][128] row-max exchange
-    static constexpr int kOffBar = kOffRed + 2 * kSplit * 128 * 4;
-    // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_empty[2], p_full, o_done, drain,
-    //           red[2], lsum
-    static constexpr int kNumBars = 1 + 4 * kStages + 4 + 3 + 3;
+    static constexpr int kOffQ = 0;                                     // [kTiles]
+    static constexpr int kOffK = kOffQ + kTiles * kQBytes;              // [kStages]
+    static constexpr int kOffV = kOffK + kStages * kKBytes;             // [kStages]
+    static constexpr int kOffP = kOffV + kStages * kVStride;            // [kTiles]
+    static constexpr int kOffQsf = kOffP + kTiles * kPBytes;            // [kTiles]
+    static constexpr int kOffKsf = kOffQsf + kTiles * kSfBytes;         // [kStages]
+    static constexpr int kOffVsf = kOffKsf + kStages * kSfBytes;        // [kStages]
+    static constexpr int kOffPsf = kOffVsf + kStages * kSfBytes;        // [kTiles]
+    static constexpr int kOffVsfConst = kOffPsf + kTiles * kSfBytes;
+    static constexpr int kOffBar = kOffVsfConst + kSfBytes;
+    // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S],
+    //           s_full[kTiles], s_loaded[kTiles], p_full[kTiles], o_done[kTiles], drain
+    static constexpr int kNumBars = 1 + 4 * kStages + 4 * kTiles + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemUsed = kOffMisc + 16;
     // >= 116 KB keeps one CTA per SM, so the 512-column TMEM allocation never waits
     static constexpr int kSmemBytes = (kSmemUsed + 1024 > 116 * 1024) ? kSmemUsed + 1024 : 116 * 1024;
 
-    // TMEM columns
-    static constexpr uint32_t kColS0 = 0;
-    static constexpr uint32_t kColS1 = T;
-    static constexpr uint32_t kColO = 2 * T;
-    static constexpr uint32_t kColQsf = (2 * T + D + 16 + 3) / 4 * 4;
-    static constexpr uint32_t kColKsf = kColQsf + 4;
-    static constexpr uint32_t kColPsf = kColKsf + 4 * kStages;
-    static constexpr uint32_t kColVsf = kColPsf + 4;
+    // TMEM columns: one S buffer shared by both tiles, then O per tile, then scale factors
+    static constexpr uint32_t kColS = 0;
+    static constexpr uint32_t kColO = T;  // + t * kOCols
+    static constexpr uint32_t kColQsf = (T + kTiles * kOCols + 3) / 4 * 4;  // + 4 t
+    static constexpr uint32_t kColKsf = kColQsf + 4 * kTiles;               // + 4 s
+    static constexpr uint32_t kColPsf = kColKsf + 4 * kStages;              // + 4 t
+    static constexpr uint32_t kColVsf = kColPsf + 4 * kTiles;               // + 8 s
     static constexpr uint32_t kColsUsed = kColVsf + 8 * kStages;
     static_assert(kColsUsed <= 512, "TMEM budget");
+    static_assert(kSmemUsed + 1024 <= 227 * 1024, "shared memory budget");
 };
 
 struct KParams {
@@ -109,7 +110,7 @@ struct KParams {
     float* O;
     uint32_t* status;
     int N;
-    int ntq;     // query tiles per head
+    int nq2;     // CTAs (pairs of query tiles) per head
     int nkv;     // key tiles per head
     int groups;  // 128-row scale groups per head
     int uos;
@@ -140,6 +141,7 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                       const __grid_constant__ CUtensorMap tmV, const KParams p) {
     using C = Cfg<D, T>;
     constexpr int S = C::kStages;
+    constexpr int NT = C::kTiles;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -158,22 +160,19 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
     uint64_t* bar_k_empty = bar_k_full + S;
     uint64_t* bar_v_full = bar_k_empty + S;
     uint64_t* bar_v_empty = bar_v_full + S;
-    uint64_t* bar_s_full = bar_v_empty + S;
-    uint64_t* bar_s_empty = bar_s_full + 2;
-    uint64_t* bar_p_full = bar_s_empty + 2;
-    uint64_t* bar_o_done = bar_p_full + 1;
-    uint64_t* bar_drain = bar_o_done + 1;
-    uint64_t* bar_red = bar_drain + 1;  // [2]
-    uint64_t* bar_lsum = bar_red + 2;
-    float* red = reinterpret_cast<float*>(smem + C::kOffRed);
+    uint64_t* bar_s_full = bar_v_empty + S;      // [NT]
+    uint64_t* bar_s_loaded = bar_s_full + NT;    // [NT]
+    uint64_t* bar_p_full = bar_s_loaded + NT;    // [NT]
+    uint64_t* bar_o_done = bar_p_full + NT;      // [NT]
+    uint64_t* bar_drain = bar_o_done + NT;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int bh = blockIdx.x / p.ntq;
-    const int qt = blockIdx.x % p.ntq;
+    const int bh = blockIdx.x / p.nq2;
+    const int qp = blockIdx.x % p.nq2;  // pair index: rows [256 qp, 256 qp + 256)
     const int nkv = p.nkv;
 
     if (tid == 0) {
@@ -184,14 +183,12 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
             mbar_init(bar_v_full + s, 1);
             mbar_init(bar_v_empty + s, 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(bar_s_full + b, 1);
-            mbar_init(bar_s_empty + b, C::kSoftThreads);
-            mbar_init(bar_red + b, C::kSoftThreads);
+        for (int t = 0; t < NT; ++t) {
+            mbar_init(bar_s_full + t, 1);
+            mbar_init(bar_s_loaded + t, 128);
+            mbar_init(bar_p_full + t, 128);
+            mbar_init(bar_o_done + t, 1);
         }
-        mbar_init(bar_lsum, C::kSoftThreads);
-        mbar_init(bar_p_full, C::kSoftThreads);
-        mbar_init(bar_o_done, 1);
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -219,9 +216,13 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int k_issued = 0, v_issued = 0;
-            mbar_arrive_expect_tx(bar_q, C::kQBytes + C::kSfBytes);
-            tma_load_3d(sQ, &tmQ, bar_q, 0, qt * 128, bh);
-            bulk_load(sQsf, p.q_sf + (static_cast<size_t>(bh) * p.groups + qt) * 512, 512, bar_q);
+            mbar_arrive_expect_tx(bar_q, NT * (C::kQBytes + C::kSfBytes));
+            for (int t = 0; t < NT; ++t) {
+                const int g = 2 * qp + t;  // 128-row group of tile t (may lie past N: zero-filled)
+                tma_load_3d(sQ + t * C::kQBytes, &tmQ, bar_q, 0, g * 128, bh);
+                const int gs = g < p.groups ? g : p.groups - 1;  // keep the scale copy inside the buffer
+                bulk_load(sQsf + t * 512, p.q_sf + (static_cast<size_t>(bh) * p.groups + gs) * 512, 512, bar_q);
+            }
             for (int j = 0; j < nkv; ++j) {
                 const int s = j % S;
                 const uint32_t n = j / S;
@@ -243,72 +244,82 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
             }
             // Drain: every copy this thread issued must land before the CTA exits.
             // On the normal path these phases completed long ago and the waits return at once.
-            {
-                int dummy = 0;
-                volatile int* no_abort = &dummy;
-                mbar_wait_bounded(bar_q, 0, no_abort, p.status, kTimeoutCode, kTimeoutNs);
-                // only the newest tile of each stage can still be in flight
-                for (int j = k_issued - S < 0 ? 0 : k_issued - S; j < k_issued; ++j)
-                    mbar_wait_bounded(bar_k_full + j % S, (j / S) & 1, no_abort, p.status, kTimeoutCode, kTimeoutNs);
-                for (int j = v_issued - S < 0 ? 0 : v_issued - S; j < v_issued; ++j)
-                    mbar_wait_bounded(bar_v_full + j % S, (j / S) & 1, no_abort, p.status, kTimeoutCode, kTimeoutNs);
-            }
+            int dummy = 0;
+            volatile int* no_abort = &dummy;
+            mbar_wait_bounded(bar_q, 0, no_abort, p.status, kTimeoutCode, kTimeoutNs);
+            // only the newest tile of each stage can still be in flight
+            for (int j = k_issued - S < 0 ? 0 : k_issued - S; j < k_issued; ++j)
+                mbar_wait_bounded(bar_k_full + j % S, (j / S) & 1, no_abort, p.status, kTimeoutCode, kTimeoutNs);
+            for (int j = v_issued - S < 0 ? 0 : v_issued - S; j < v_issued; ++j)
+                mbar_wait_bounded(bar_v_full + j % S, (j / S) & 1, no_abort, p.status, kTimeoutCode, kTimeoutNs);
         }
     } else if (warp == C::kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t t_s[2] = {tbase + C::kColS0, tbase + C::kColS1};
-            const uint32_t t_o = tbase + C::kColO;
-            const uint64_t qdesc = smem_desc(smem_u32(sQ), 16, C::kQKSbo, C::kQKLayout);
-            const uint64_t pdesc = smem_desc(smem_u32(sP), 16, C::kPVSbo, C::kPVLayout);
-            bool ok = mbar_wait_bounded(bar_q, 0, abort_flag, p.status, kTimeoutCode, kTimeoutNs);
-            if (ok) {
-                tc_fence_after_sync();
-                tc_cp_sf(tbase + C::kColQsf, sf_desc(sQsf));
-                if (D == 128)
-                    for (int s = 0; s < S; ++s) tc_cp_sf(tbase + C::kColVsf + 8 * s + 4, sf_desc(sVsfConst));
-            }
-            auto issue_s = [&](int j) -> bool {
+            const uint32_t t_s = tbase + C::kColS;
+            auto wait = [&](uint64_t* bar, uint32_t parity) {
+                return mbar_wait_bounded(bar, parity, abort_flag, p.status, kTimeoutCode, kTimeoutNs);
+            };
+            // S_t(j) = Q_t K(j)^T into the shared S buffer.  Tile A's issue also
+            // waits for K(j) and copies its scales; tile B reuses both.
+            auto issue_s = [&](int t, int j) -> bool {
                 const int s = j % S;
                 const uint32_t n = j / S;
-                const int b = j & 1;
-                if (!mbar_wait_bounded(bar_k_full + s, n & 1, abort_flag, p.status, kTimeoutCode, kTimeoutNs))
-                    return false;
-                if (j >= 2 && !mbar_wait_bounded(bar_s_empty + b, ((j - 2) >> 1) & 1, abort_flag, p.status,
-                                                 kTimeoutCode, kTimeoutNs))
-                    return false;
-                tc_fence_after_sync();
-                tc_cp_sf(tbase + C::kColKsf + 4 * s, sf_desc(sKsf + s * 512));
+                if (t == 0) {
+                    if (!wait(bar_k_full + s, n & 1)) return false;
+                    tc_fence_after_sync();
+                    tc_cp_sf(tbase + C::kColKsf + 4 * s, sf_desc(sKsf + s * 512));
+                }
+                const uint64_t qdesc = smem_desc(smem_u32(sQ + t * C::kQBytes), 16, C::kQKSbo, C::kQKLayout);
                 const uint64_t kdesc = smem_desc(smem_u32(sK + s * C::kKBytes), 16, C::kQKSbo, C::kQKLayout);
                 const uint32_t ksf = tbase + C::kColKsf + 4 * s + ((T == 64) ? 2 * (j & 1) : 0);
 #pragma unroll
                 for (int kk = 0; kk < D / 64; ++kk)
-                    tc_mma_mxf4(t_s[b], qdesc + 2 * kk, kdesc + 2 * kk, mxf4_idesc(T, 2 * kk, 2 * kk),
-                                tbase + C::kColQsf, ksf, kk > 0 ? 1u : 0u);
-                tc_commit(bar_s_full + b);
-                tc_commit(bar_k_empty + s);
+                    tc_mma_mxf4(t_s, qdesc + 2 * kk, kdesc + 2 * kk, mxf4_idesc(T, 2 * kk, 2 * kk),
+                                tbase + C::kColQsf + 4 * t, ksf, kk > 0 ? 1u : 0u);
+                tc_commit(bar_s_full + t);
+                if (t == NT - 1) tc_commit(bar_k_empty + s);
                 return true;
             };
-            if (ok) ok = issue_s(0);
-            for (int j = 0; ok && j < nkv; ++j) {
-                if (j + 1 < nkv && !issue_s(j + 1)) break;
+            // O_t += P_t V(j).  Tile A's issue waits for V(j) and copies its scales.
+            auto issue_pv = [&](int t, int j) -> bool {
                 const int s = j % S;
                 const uint32_t n = j / S;
-                if (!mbar_wait_bounded(bar_p_full, j & 1, abort_flag, p.status, kTimeoutCode, kTimeoutNs)) break;
-                if (!mbar_wait_bounded(bar_v_full + s, n & 1, abort_flag, p.status, kTimeoutCode, kTimeoutNs))
-                    break;
+                if (!wait(bar_p_full + t, j & 1)) return false;
+                if (t == 0 && !wait(bar_v_full + s, n & 1)) return false;
                 tc_fence_after_sync();
-                tc_cp_sf(tbase + C::kColPsf, sf_desc(sPsf));
-                tc_cp_sf(tbase + C::kColVsf + 8 * s, sf_desc(sVsf + s * 512));
+                tc_cp_sf(tbase + C::kColPsf + 4 * t, sf_desc(sPsf + t * 512));
+                if (t == 0) tc_cp_sf(tbase + C::kColVsf + 8 * s, sf_desc(sVsf + s * 512));
+                const uint64_t pdesc = smem_desc(smem_u32(sP + t * C::kPBytes), 16, C::kPVSbo, C::kPVLayout);
                 const uint64_t vdesc = smem_desc(smem_u32(sV + s * C::kVStride), 16, C::kPVSbo, C::kPVLayout);
 #pragma unroll
                 for (int kk = 0; kk < T / 64; ++kk) {
                     const uint32_t sfb_id = (T == 64) ? 2u * (j & 1) : 2u * kk;
-                    tc_mma_mxf4(t_o, pdesc + 2 * kk, vdesc + 2 * kk, mxf4_idesc(D + 16, 2 * kk, sfb_id),
-                                tbase + C::kColPsf, tbase + C::kColVsf + 8 * s, (j > 0 || kk > 0) ? 1u : 0u);
+                    tc_mma_mxf4(tbase + C::kColO + t * C::kOCols, pdesc + 2 * kk, vdesc + 2 * kk,
+                                mxf4_idesc(D + 16, 2 * kk, sfb_id), tbase + C::kColPsf + 4 * t,
+                                tbase + C::kColVsf + 8 * s, (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                tc_commit(bar_v_empty + s);
-                tc_commit(bar_o_done);
+                tc_commit(bar_o_done + t);
+                if (t == NT - 1) tc_commit(bar_v_empty + s);
+                return true;
+            };
+            bool ok = wait(bar_q, 0);
+            if (ok) {
+                tc_fence_after_sync();
+                for (int t = 0; t < NT; ++t) tc_cp_sf(tbase + C::kColQsf + 4 * t, sf_desc(sQsf + t * 512));
+                if (D == 128)
+                    for (int s = 0; s < S; ++s) tc_cp_sf(tbase + C::kColVsf + 8 * s + 4, sf_desc(sVsfConst));
+            }
+            // Order: S_A(0); S_B(0) after A loaded; S_A(1) after B loaded; then per tile j:
+            // PV_A(j), S_B(j+1) (after A loaded S_A(j+1)), PV_B(j), S_A(j+2) (after B loaded S_B(j+1)).
+            ok = ok && issue_s(0, 0);
+            ok = ok && wait(bar_s_loaded + 0, 0) && issue_s(1, 0);
+            if (nkv > 1) ok = ok && wait(bar_s_loaded + 1, 0) && issue_s(0, 1);
+            for (int j = 0; ok && j < nkv; ++j) {
+                if (!issue_pv(0, j)) break;
+                if (j + 1 < nkv && !(wait(bar_s_loaded + 0, (j + 1) & 1) && issue_s(1, j + 1))) break;
+                if (!issue_pv(1, j)) break;
+                if (j + 2 < nkv && !(wait(bar_s_loaded + 1, (j + 1) & 1) && issue_s(0, j + 2))) break;
             }
             // Drain: wait for every MMA / copy this thread issued before TMEM is freed.
             tc_commit(bar_drain);
@@ -316,78 +327,58 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
             mbar_wait_bounded(bar_drain, 0, &dummy, p.status, kTimeoutCode, kTimeoutNs);
         }
     } else {
-        // ------------------------------------------------------------ softmax
-        // kSplit threads per query row (= TMEM lane): thread `part` owns S columns
-        // [part*kCols, (part+1)*kCols) of every tile, i.e. kBlk 32-column P blocks.
-        constexpr int kCols = C::kCols;
-        constexpr int kBlk = C::kBlk;
+        // ------------------------------------------------------------ softmax (thread = query row of tile t)
+        const int t = warp >> 2;
         const int row = tid & 127;
-        const int part = tid >> 7;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t t_o = tbase + lane_base + C::kColO + t * C::kOCols;
         const float kq = p.kq;
         const int uos = p.uos;
         const int valid_last = p.N - (nkv - 1) * T;
+        uint8_t* sPt = sP + t * C::kPBytes;
+        uint8_t* sPsft = sPsf + t * 512;
         float m_run = -INFINITY;
-        float l_run = 0.f;  // PNQ off: this thread's share of the row sum
+        float l_run = 0.f;  // PNQ off: the row sum of the unquantized exponentials
         bool ok = true;
         for (int j = 0; j < nkv; ++j) {
-            const int b = j & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_s_full + b, (j >> 1) & 1, abort_flag, p.status,
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_s_full + t, j & 1, abort_flag, p.status,
                                                             kTimeoutCode, kTimeoutNs))) {
                 ok = false;
                 break;
             }
             tc_fence_after_sync();
-            float sv[kCols];
-            {
-                const uint32_t taddr = tbase + lane_base + (b ? C::kColS1 : C::kColS0) + part * kCols;
-                if constexpr (kCols == 64) {
-                    uint32_t r[64];
-                    tmem_ld64_sync(taddr, r);
+            float sv[T];
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) sv[i] = __uint_as_float(r[i]);
-                } else {
-                    uint32_t r[32];
-                    tmem_ld32_sync(taddr, r);
+            for (int c = 0; c < T / 64; ++c) {
+                uint32_t r[64];
+                tmem_ld64_sync(tbase + lane_base + C::kColS + 64 * c, r);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(r[i]);
-                }
+                for (int i = 0; i < 64; ++i) sv[64 * c + i] = __uint_as_float(r[i]);
             }
             tc_fence_before_sync();
-            mbar_arrive(bar_s_empty + b);
+            mbar_arrive(bar_s_loaded + t);
             if (j == nkv - 1 && valid_last < T) {
 #pragma unroll
-                for (int i = 0; i < kCols; ++i)
-                    if (part * kCols + i >= valid_last) sv[i] = -INFINITY;
+                for (int i = 0; i < T; ++i)
+                    if (i >= valid_last) sv[i] = -INFINITY;
             }
-            float bm[kBlk];
+            float bm[T / 32];
 #pragma unroll
-            for (int k = 0; k < kBlk; ++k) bm[k] = block_max32(sv + 32 * k);
-            float lmax = bm[0];
+            for (int k = 0; k < T / 32; ++k) bm[k] = block_max32(sv + 32 * k);
+            float tmax = bm[0];
 #pragma unroll
-            for (int k = 1; k < kBlk; ++k) lmax = fmaxf(lmax, bm[k]);
-            // exchange the partial maxima of the row's kSplit threads
-            red[(b * C::kSplit + part) * 128 + row] = lmax;
-            mbar_arrive(bar_red + b);
-            if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_red + b, (j >> 1) & 1, abort_flag, p.status,
-                                                            kTimeoutCode, kTimeoutNs))) {
-                ok = false;
-                break;
-            }
-            float tmax = red[(b * C::kSplit) * 128 + row];
-#pragma unroll
-            for (int q = 1; q < C::kSplit; ++q) tmax = fmaxf(tmax, red[(b * C::kSplit + q) * 128 + row]);
+            for (int k = 1; k < T / 32; ++k) tmax = fmaxf(tmax, bm[k]);
             const float m_new = fmaxf(m_run, tmax);
             const bool rescale = (j > 0) && (m_new > m_run);
             const float alpha = rescale ? ex2_approx((m_run - m_new) * kq) : 1.f;
 
             // PNQ: quantize exp(S - m_new) per 32-column block.  pmax = 2^((bm - m) * kq)
             // gives the block exponent e; each element is then 2^(s*kq - (m*kq + e)).
-            uint32_t pw[kCols / 8];
+            uint32_t pw[T / 8];
             uint32_t sfw = 0;
             float lsum = 0.f;
 #pragma unroll
-            for (int k = 0; k < kBlk; ++k) {
+            for (int k = 0; k < T / 32; ++k) {
                 const float pmax = ex2_approx((bm[k] - m_new) * kq);
                 const int e = block_exponent_f32(__float_as_uint(pmax), uos);
                 const float nbias = -fmaf(m_new, kq, static_cast<float>(e));
@@ -411,9 +402,9 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                 sfw |= static_cast<uint32_t>(e + 127) << (8 * k);
                 if constexpr (!PNQ) lsum = fmaf(bsum, exp2_neg_int(-e), lsum);
             }
-            // The P buffer and O are free once the previous P*V finished.
+            // The P buffer and O are free once the previous P*V of this tile finished.
             if (j > 0) {
-                if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_o_done, (j - 1) & 1, abort_flag, p.status,
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_o_done + t, (j - 1) & 1, abort_flag, p.status,
                                                                 kTimeoutCode, kTimeoutNs))) {
                     ok = false;
                     break;
@@ -421,84 +412,56 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                 tc_fence_after_sync();
             }
             if (__any_sync(0xffffffffu, rescale)) {
-                // this thread's share of O's columns (part 0 also owns the row-sum columns under PNQ)
-                constexpr int kOCols = D / C::kSplit;
-                const uint32_t obase = tbase + lane_base + C::kColO + part * kOCols;
 #pragma unroll
-                for (int c = 0; c < kOCols / 32; ++c) {
+                for (int c = 0; c < D / 32; ++c) {
                     uint32_t r[32];
-                    tmem_ld32_sync(obase + 32 * c, r);
+                    tmem_ld32_sync(t_o + 32 * c, r);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st32(obase + 32 * c, r);
+                    tmem_st32(t_o + 32 * c, r);
                 }
-                if (PNQ && part == 0) {
-                    uint32_t r[16];
-                    tmem_ld16_sync(tbase + lane_base + C::kColO + D, r);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st16(tbase + lane_base + C::kColO + D, r);
+                if constexpr (PNQ) {
+                    const uint32_t lcol = __float_as_uint(__uint_as_float(tmem_ld1_sync(t_o + D)) * alpha);
+                    uint32_t r[16] = {lcol};
+                    tmem_st16(t_o + D, r);  // columns D+1.. are zero (zero V^T rows)
                 }
                 tmem_st_wait();
             }
-            // P row share -> shared memory in the swizzled K-major layout the MMA reads.
+            // P row -> shared memory in the swizzled K-major layout the MMA reads.
             {
-                uint8_t* prow = sP + row * (T / 2);
+                uint8_t* prow = sPt + row * (T / 2);
 #pragma unroll
-                for (int k = 0; k < kBlk; ++k) {
-                    const int c = part * kBlk + k;  // 16-byte chunk = one 32-column block
+                for (int c = 0; c < T / 32; ++c) {
                     const int phys = (T == 128) ? (c ^ ((row >> 1) & 3)) : (c ^ ((row >> 2) & 1));
                     *reinterpret_cast<uint4*>(prow + 16 * phys) =
-                        make_uint4(pw[4 * k], pw[4 * k + 1], pw[4 * k + 2], pw[4 * k + 3]);
+                        make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
                 }
-                uint8_t* sfp = sPsf + (row & 31) * 16 + (row >> 5) * 4 + part * kBlk;
-                if constexpr (kBlk == 2)
-                    *reinterpret_cast<uint16_t*>(sfp) = static_cast<uint16_t>(sfw);
-                else if constexpr (kBlk == 1)
-                    *sfp = static_cast<uint8_t>(sfw);
-                else
-                    *reinterpret_cast<uint32_t*>(sfp) = sfw;
+                reinterpret_cast<uint32_t*>(sPsft)[(row & 31) * 4 + (row >> 5)] = sfw;
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
-            mbar_arrive(bar_p_full);
+            mbar_arrive(bar_p_full + t);
             if constexpr (!PNQ) l_run = fmaf(l_run, alpha, lsum);
             m_run = m_new;
         }
         // Epilogue: O / l for the valid rows.
-        if (ok && __all_sync(0xffffffffu, mbar_wait_bounded(bar_o_done, (nkv - 1) & 1, abort_flag, p.status,
+        if (ok && __all_sync(0xffffffffu, mbar_wait_bounded(bar_o_done + t, (nkv - 1) & 1, abort_flag, p.status,
                                                              kTimeoutCode, kTimeoutNs))) {
             tc_fence_after_sync();
-            float l;
-            bool have_l = true;
-            if constexpr (PNQ) {
-                l = __uint_as_float(tmem_ld1_sync(tbase + lane_base + C::kColO + D));
-            } else {
-                red[part * 128 + row] = l_run;  // the exchange buffers are idle after the loop
-                mbar_arrive(bar_lsum);
-                have_l = __all_sync(0xffffffffu, mbar_wait_bounded(bar_lsum, 0, abort_flag, p.status,
-                                                                   kTimeoutCode, kTimeoutNs));
-                l = 0.f;
+            const float l = PNQ ? __uint_as_float(tmem_ld1_sync(t_o + D)) : l_run;
+            const float inv_l = 1.f / l;
+            const int qrow = qp * C::kRows + t * 128 + row;
+            float* out = p.O + (static_cast<size_t>(bh) * p.N + qrow) * D;
 #pragma unroll
-                for (int q = 0; q < C::kSplit; ++q) l += red[q * 128 + row];
-            }
-            if (have_l) {
-                const float inv_l = 1.f / l;
-                const int qrow = qt * 128 + row;
-                constexpr int kOCols = D / C::kSplit;
-                float* out = p.O + (static_cast<size_t>(bh) * p.N + qrow) * D + part * kOCols;
-                const uint32_t obase = tbase + lane_base + C::kColO + part * kOCols;
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32_sync(t_o + 32 * c, r);
+                if (qrow < p.N) {
 #pragma unroll
-                for (int c = 0; c < kOCols / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32_sync(obase + 32 * c, r);
-                    if (qrow < p.N) {
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4*>(out + 32 * c + i) =
-                                make_float4(__uint_as_float(r[i]) * inv_l, __uint_as_float(r[i + 1]) * inv_l,
-                                            __uint_as_float(r[i + 2]) * inv_l, __uint_as_float(r[i + 3]) * inv_l);
-                    }
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4*>(out + 32 * c + i) =
+                            make_float4(__uint_as_float(r[i]) * inv_l, __uint_as_float(r[i + 1]) * inv_l,
+                                        __uint_as_float(r[i + 2]) * inv_l, __uint_as_float(r[i + 3]) * inv_l);
                 }
             }
         }
@@ -563,12 +526,12 @@ cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
     kp.O = a.O;
     kp.status = a.status;
     kp.N = a.N;
-    kp.ntq = (a.N + 127) / 128;
+    kp.nq2 = (a.N + C::kRows - 1) / C::kRows;
     kp.nkv = (a.N + T - 1) / T;
     kp.groups = (a.N + 127) / 128;
     kp.uos = a.uos;
     kp.kq = static_cast<float>(static_cast<double>(a.softmax_scale) * 1.4426950408889634);
-    dim3 grid(static_cast<unsigned>(a.BH * kp.ntq));
+    dim3 grid(static_cast<unsigned>(a.BH * kp.nq2));
     mxattn_fwd_kernel<D, T, PNQ><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, kp);
     return cudaGetLastError();
 }
