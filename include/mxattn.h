@@ -149,6 +149,33 @@ mxattn_status mxattn_forward_quantized(const uint8_t* q_codes, const uint8_t* q_
                                        mxattn_stream_t stream);
 
 /*
+ * mxattn_forward without a caller-provided workspace, for callers that cannot
+ * allocate device memory themselves: code embedded in a host framework that
+ * owns all device memory through its own pool and forbids raw cudaMalloc, or
+ * a latency-critical loop that must not pay for cudaMalloc's implicit device
+ * synchronization.  (The MXAttention paper has no counterpart; this is a
+ * deployment convenience.)
+ *   - The workspace is a fixed 16 MiB array of device memory inside this
+ *     library's CUDA module; every device that loads the library holds it
+ *     until the process exits.  Shapes whose mxattn_workspace_size exceeds
+ *     16 MiB (16777216 bytes) are rejected with MXATTN_ERR_UNSUPPORTED before
+ *     anything is launched.  The call itself allocates and frees nothing.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device); make that first call before any stream capture.
+ *   - All calls share the one array, and it keeps the last call's contents
+ *     (each call rewrites what it reads, including the status word).  Calls
+ *     that may overlap on the GPU -- on different streams, or from different
+ *     threads -- race on it; serialize them.
+ *   - The kernels' timeout status is not reported by this call (a bounded
+ *     wait that gives up leaves O unspecified); use mxattn_forward with a
+ *     workspace and mxattn_workspace_status when that status is needed.
+ * Arguments, constraints and other errors as mxattn_forward.
+ */
+mxattn_status mxattn_forward_noalloc(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                     int kv_tile, int pnq, mxattn_rule rule, float softmax_scale, float* O,
+                                     mxattn_stream_t stream);
+
+/*
  * Synchronizes `stream`, reads the status word of `workspace` (written by
  * the last forward that used it) and returns MXATTN_OK or
  * MXATTN_ERR_TIMEOUT.  MXATTN_ERR_CUDA if the synchronization or copy fails.

@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.mxattn_forward_quantized.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
                                                ctypes.c_float, P, P, u64, P]
         L.mxattn_forward_quantized.restype = i32
+        L.mxattn_forward_noalloc.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, ctypes.c_float, P, P]
+        L.mxattn_forward_noalloc.restype = i32
         L.mxattn_workspace_status.argtypes = [P, P]
         L.mxattn_workspace_status.restype = i32
         _lib = L
@@ -205,6 +207,26 @@ def mxattn_forward_quantized(q_codes, q_scales, k_codes, k_scales, vt_codes, vt_
         _cuda(k_scales, "k_scales"), _cuda(vt_codes, "vt_codes"), _cuda(vt_scales, "vt_scales"),
         B, H, N, d, kv_tile, 1 if pnq else 0, _rule(rule), float(softmax_scale), _cuda(out, "out", torch.float32),
         _cuda(workspace, "workspace"), workspace.numel(), _stream(stream)), "mxattn_forward_quantized")
+    return out
+
+
+NOALLOC_MAX_WORKSPACE = 16 << 20  # bytes of the library's fixed scratch (include/mxattn.h)
+
+
+def mxattn_forward_noalloc(q, k, v, kv_tile=128, pnq=True, rule="uos", softmax_scale=0.0, out=None, stream=None):
+    """mxattn_forward on the library's fixed scratch: no workspace argument and no
+    device allocation inside the call (the output tensor is still the caller's).
+    For callers that cannot allocate device memory; shapes whose workspace exceeds
+    16 MiB are rejected.  Calls that overlap on the GPU race on the shared scratch."""
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
+    _check(lib().mxattn_forward_noalloc(_cuda(q, "q", torch.bfloat16), _cuda(k, "k", torch.bfloat16),
+                                        _cuda(v, "v", torch.bfloat16), B, H, N, d, kv_tile, 1 if pnq else 0,
+                                        _rule(rule), float(softmax_scale), _cuda(out, "out", torch.float32),
+                                        _stream(stream)), "mxattn_forward_noalloc")
     return out
 
 
