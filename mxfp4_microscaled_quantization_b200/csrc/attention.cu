@@ -10,8 +10,9 @@
 // walks all key tiles in ascending order; both tiles share every K / V^T tile
 // and one TMEM buffer for S, and their softmax warpgroups run a half-step
 // apart (ping-pong), so one tile's serial phases (TMEM load, waits, O
-// rescale, P hand-off) overlap the other tile's exponentials.  Roles (320
-// threads):
+// rescale, P hand-off) overlap the other tile's exponentials.  Roles (384
+// threads, three warpgroups; setmaxnreg gives the two softmax warpgroups 224
+// registers per thread and the third 56):
 //   warps 0-3 / 4-7    softmax for tile A / B, one thread per query row (=
 //                      TMEM lane): running max, exp2 on the MUFU with packed
 //                      f32x2 FMAs, per-32-column block exponent (UOS/OCP),
@@ -23,6 +24,7 @@
 //                      tcgen05.mma kind::mxf4 block_scale, in the order
 //                      S_A(j), S_B(j), S_A(j+1) ... interleaved with
 //                      O_A += P_A V(j), O_B += P_B V(j).
+//   warps 10-11        idle (they complete the third warpgroup).
 // The row sum under PNQ is produced by the tensor core itself: V^T gets one
 // extra row of ones (E2M1 1.0, scale 2^0) so O's column d accumulates
 // sum_j q_j -- exactly the quantized values that multiply V -- and is
@@ -48,6 +50,14 @@ namespace {
 
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
 constexpr uint32_t kTimeoutCode = 4u;           // MXATTN_ERR_TIMEOUT
+#ifndef MXATTN_FMA_EXP_PAIRS
+#define MXATTN_FMA_EXP_PAIRS 1
+#endif
+#ifndef MXATTN_ROLE_WAIT_HINT_NS
+#define MXATTN_ROLE_WAIT_HINT_NS 0
+#endif
+// Suspend hint for the producer's and the MMA issuer's waits (0: plain try_wait).
+constexpr uint32_t kRoleWaitHintNs = MXATTN_ROLE_WAIT_HINT_NS;
 
 template <int D, int T>
 struct Cfg {
@@ -57,7 +67,16 @@ struct Cfg {
     static constexpr int kSoftThreads = 128 * kTiles;
     static constexpr int kProducerWarp = 4 * kTiles;
     static constexpr int kMmaWarp = 4 * kTiles + 1;
-    static constexpr int kThreads = kSoftThreads + 64;
+    // A third, full warpgroup holds the producer and MMA warps (plus two idle
+    // warps) so registers can move between warpgroups with setmaxnreg.
+    static constexpr int kThreads = kSoftThreads + 128;
+    // Launch: kThreads x kLaunchRegs registers (ptxas's cap for 12 warps, 3 per
+    // sub-partition).  Split: softmax warpgroups kSoftRegs, the other kRoleRegs;
+    // 2 x 128 x 224 + 128 x 56 == 384 x 168.
+    static constexpr uint32_t kLaunchRegs = 168;
+    static constexpr uint32_t kSoftRegs = 224;
+    static constexpr uint32_t kRoleRegs = 56;
+    static_assert(kTiles * 128 * kSoftRegs + 128 * kRoleRegs == kThreads * kLaunchRegs, "register split");
     static constexpr int kQBytes = 128 * D / 2;
     static constexpr int kKBytes = T * D / 2;
     static constexpr int kVRows = D + 16;  // V^T rows + a row of ones + 15 zero rows
@@ -66,6 +85,7 @@ struct Cfg {
     static constexpr int kPBytes = 128 * T / 2;
     static constexpr int kSfBytes = 512;
     static constexpr int kOCols = D + 16;
+    static constexpr int kFmaExpPairs = MXATTN_FMA_EXP_PAIRS;  // of every 4 exponential pairs, this many use the FMA pipe
 
     static constexpr uint32_t kQKLayout = (D == 128) ? kLayoutSw64 : kLayoutSw32;
     static constexpr uint32_t kQKSbo = 8 * D / 2;
@@ -212,7 +232,12 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
     tc_fence_after_sync();
     const uint32_t tbase = *tmem_holder;
 
-    if (warp == C::kProducerWarp) {
+    // Each warpgroup's code lives entirely in its own branch (register budget
+    // set by setmaxnreg at the top of the branch), ending with a block-wide
+    // named barrier after which the MMA warp frees TMEM.
+    if (warp >= 4 * NT) {
+        warpgroup_regs_dec<C::kRoleRegs>();
+        if (warp == C::kProducerWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int k_issued = 0, v_issued = 0;
@@ -228,14 +253,14 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                 const uint32_t n = j / S;
                 const size_t grp = static_cast<size_t>(bh) * p.groups + (j * T) / 128;
                 if (j >= S && !mbar_wait_bounded(bar_k_empty + s, (n - 1) & 1, abort_flag, p.status, kTimeoutCode,
-                                                 kTimeoutNs))
+                                                 kTimeoutNs, kRoleWaitHintNs))
                     break;
                 mbar_arrive_expect_tx(bar_k_full + s, C::kKBytes + C::kSfBytes);
                 tma_load_3d(sK + s * C::kKBytes, &tmK, bar_k_full + s, 0, j * T, bh);
                 bulk_load(sKsf + s * 512, p.k_sf + grp * 512, 512, bar_k_full + s);
                 k_issued = j + 1;
                 if (j >= S && !mbar_wait_bounded(bar_v_empty + s, (n - 1) & 1, abort_flag, p.status, kTimeoutCode,
-                                                 kTimeoutNs))
+                                                 kTimeoutNs, kRoleWaitHintNs))
                     break;
                 mbar_arrive_expect_tx(bar_v_full + s, C::kVLoadBytes + C::kSfBytes);
                 tma_load_3d(sV + s * C::kVStride, &tmV, bar_v_full + s, j * (T / 2), 0, bh);
@@ -258,7 +283,7 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
         if (lane == 0) {
             const uint32_t t_s = tbase + C::kColS;
             auto wait = [&](uint64_t* bar, uint32_t parity) {
-                return mbar_wait_bounded(bar, parity, abort_flag, p.status, kTimeoutCode, kTimeoutNs);
+                return mbar_wait_bounded(bar, parity, abort_flag, p.status, kTimeoutCode, kTimeoutNs, kRoleWaitHintNs);
             };
             // S_t(j) = Q_t K(j)^T into the shared S buffer.  Tile A's issue also
             // waits for K(j) and copies its scales; tile B reuses both.
@@ -326,7 +351,15 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
             int dummy = 0;
             mbar_wait_bounded(bar_drain, 0, &dummy, p.status, kTimeoutCode, kTimeoutNs);
         }
+    }
+    tc_fence_before_sync();
+    named_barrier_sync(1, C::kThreads);
+    if (warp == C::kMmaWarp) {
+        tc_fence_after_sync();
+        tmem_dealloc(tbase, 512);
+    }
     } else {
+        warpgroup_regs_inc<C::kSoftRegs>();
         // ------------------------------------------------------------ softmax (thread = query row of tile t)
         const int t = warp >> 2;
         const int row = tid & 127;
@@ -390,8 +423,12 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                     for (int i = 0; i < 8; i += 2) {
                         float w0, w1;
                         ffma2_bcast(w0, w1, sv[32 * k + 8 * g + i], sv[32 * k + 8 * g + i + 1], kq, nbias);
-                        f[i] = ex2_approx(w0);
-                        f[i + 1] = ex2_approx(w1);
+                        if (i / 2 < 4 - C::kFmaExpPairs) {  // MUFU
+                            f[i] = ex2_approx(w0);
+                            f[i + 1] = ex2_approx(w1);
+                        } else {                            // FMA pipe
+                            exp2_fma_x2(w0, w1, f[i], f[i + 1]);
+                        }
                     }
                     if constexpr (!PNQ) {
 #pragma unroll
@@ -413,18 +450,15 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
             }
             if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32_sync(t_o + 32 * c, r);
+                for (int c = 0; c < D / 64; ++c) {
+                    uint32_t r[64];
+                    tmem_ld64_sync(t_o + 64 * c, r);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st32(t_o + 32 * c, r);
+                    for (int i = 0; i < 64; i += 2) fmul2_bcast(r[i], r[i + 1], r[i], r[i + 1], alpha);
+                    tmem_st64(t_o + 64 * c, r);
                 }
-                if constexpr (PNQ) {
-                    const uint32_t lcol = __float_as_uint(__uint_as_float(tmem_ld1_sync(t_o + D)) * alpha);
-                    uint32_t r[16] = {lcol};
-                    tmem_st16(t_o + D, r);  // columns D+1.. are zero (zero V^T rows)
-                }
+                if constexpr (PNQ)
+                    tmem_st1(t_o + D, __float_as_uint(__uint_as_float(tmem_ld1_sync(t_o + D)) * alpha));
                 tmem_st_wait();
             }
             // P row -> shared memory in the swizzled K-major layout the MMA reads.
@@ -465,13 +499,8 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                 }
             }
         }
-    }
-
-    tc_fence_before_sync();
-    __syncthreads();
-    if (warp == C::kMmaWarp) {
-        tc_fence_after_sync();
-        tmem_dealloc(tbase, 512);
+        tc_fence_before_sync();
+        named_barrier_sync(1, C::kThreads);
     }
 }
 
@@ -508,8 +537,14 @@ cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
     using C = Cfg<D, T>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, T, PNQ>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        // The setmaxnreg split assumes the launch allocates exactly kLaunchRegs per
+        // thread; with fewer, the softmax warpgroups' increase could never be met.
+        cudaFuncAttributes fa{};
+        cudaError_t e = cudaFuncGetAttributes(&fa, mxattn_fwd_kernel<D, T, PNQ>);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != static_cast<int>(C::kLaunchRegs)) return cudaErrorInvalidConfiguration;
+        e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, T, PNQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }

@@ -48,16 +48,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
+// try_wait that lets the hardware suspend the thread for up to `hint_ns`
+// while the phase is incomplete (it resumes as soon as the phase completes).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return done != 0;
+}
+
 // Wait for the phase with the given parity to complete, giving up after
 // `timeout_ns` of wall time or as soon as another role of the CTA raised
 // `*abort_flag`.  On timeout it raises the flag and ORs `code` into the
 // global status word.  Returns false when the wait gave up.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                                  uint32_t* status, uint32_t code, uint64_t timeout_ns) {
+                                                  uint32_t* status, uint32_t code, uint64_t timeout_ns,
+                                                  uint32_t hint_ns = 0) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (hint_ns ? mbar_try_wait_hint(bar, parity, hint_ns) : mbar_try_wait(bar, parity)) return true;
         if ((it & 63u) == 0u) {
             if (*abort_flag) return false;
             if (global_timer_ns() - t0 > timeout_ns) {
@@ -89,6 +104,24 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Block-wide named barrier `id` over `nthreads` threads (the arrival point may
+// differ between warps).
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ------------------------------------------------------------------ register reallocation
+
+// Move registers between warpgroups (executed by every thread of a warpgroup).
+template <uint32_t kRegs>
+__device__ __forceinline__ void warpgroup_regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs>
+__device__ __forceinline__ void warpgroup_regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
 // ------------------------------------------------------------------ tcgen05
@@ -216,6 +249,10 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&v)[64
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ uint32_t tmem_ld1_sync(uint32_t taddr) {
     uint32_t v;
     asm volatile(
@@ -277,6 +314,55 @@ __device__ __forceinline__ void ffma2_bcast(float& o0, float& o1, float x0, floa
         "mov.b64 {%0, %1}, d;\n\t}"
         : "=f"(o0), "=f"(o1)
         : "f"(x0), "f"(x1), "f"(k), "f"(c));
+}
+
+
+// (o0, o1) = (x0, x1) * k as one packed f32x2 multiply.
+__device__ __forceinline__ void fmul2_bcast(uint32_t& o0, uint32_t& o1, uint32_t x0, uint32_t x1, float k) {
+    asm("{\n\t.reg .b64 a, b, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 b, {%4, %4};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "=r"(o0), "=r"(o1)
+        : "r"(x0), "r"(x1), "f"(k));
+}
+
+// 2^w for two values on the FMA pipe instead of the MUFU (Cody & Waite style
+// range reduction: 2^w = 2^n * 2^f, n = round(w), f = w - n in [-1/2, 1/2]).
+// 2^f is a degree-5 polynomial fitted for relative error on [-1/2, 1/2]
+// (coefficients from csrc/exp2_poly_fit.py; max relative error 2.3e-7 in fp32),
+// 2^n is added to the exponent field.  Inputs are clamped at -125 so the
+// result stays a normal number (2^-125 where the exact value is smaller).
+__device__ __forceinline__ void exp2_fma_x2(float w0, float w1, float& v0, float& v1) {
+    w0 = fmaxf(w0, -125.f);
+    w1 = fmaxf(w1, -125.f);
+    uint32_t p0, p1, t0, t1;
+    asm("{\n\t.reg .b64 w, t, n, f, p, c;\n\t"
+        "mov.b64 w, {%4, %5};\n\t"
+        "mov.b64 c, {%6, %6};\n\t"
+        "add.rn.f32x2 t, w, c;\n\t"      // round(w) lands in the low mantissa bits of t
+        "sub.rn.f32x2 n, t, c;\n\t"      // n = round(w)
+        "sub.rn.f32x2 f, w, n;\n\t"      // f in [-1/2, 1/2]
+        "mov.b64 p, {%12, %12};\n\t"
+        "mov.b64 c, {%11, %11};\n\t"
+        "fma.rn.f32x2 p, p, f, c;\n\t"
+        "mov.b64 c, {%10, %10};\n\t"
+        "fma.rn.f32x2 p, p, f, c;\n\t"
+        "mov.b64 c, {%9, %9};\n\t"
+        "fma.rn.f32x2 p, p, f, c;\n\t"
+        "mov.b64 c, {%8, %8};\n\t"
+        "fma.rn.f32x2 p, p, f, c;\n\t"
+        "mov.b64 c, {%7, %7};\n\t"
+        "fma.rn.f32x2 p, p, f, c;\n\t"
+        "mov.b64 {%0, %1}, p;\n\t"
+        "mov.b64 {%2, %3}, t;\n\t}"
+        : "=r"(p0), "=r"(p1), "=r"(t0), "=r"(t1)
+        : "f"(w0), "f"(w1), "f"(12582912.0f),  // 1.5 * 2^23
+          "f"(0x1.000002p+0f), "f"(0x1.62e428p-1f), "f"(0x1.ebf91ap-3f), "f"(0x1.c6b782p-5f), "f"(0x1.3d0ba4p-7f),
+          "f"(0x1.5bc922p-10f));
+    v0 = __uint_as_float(p0 + (t0 << 23));
+    v1 = __uint_as_float(p1 + (t1 << 23));
 }
 
 // ------------------------------------------------------------------ E2M1 / E8M0 helpers

@@ -39,6 +39,7 @@ def assert_close(O, R, what=""):
     rel = np.linalg.norm(O - R) / np.linalg.norm(R)
     mabs = float(np.max(np.abs(O - R)))
     assert rel <= REL_FROB and mabs <= MAX_ABS, f"{what}: rel-Frobenius {rel:.3e}, max-abs {mabs:.3e}"
+    print(f"[parity] {what}: rel-Frobenius {rel:.3e}, max-abs {mabs:.3e}")
     return rel, mabs
 
 
