@@ -30,7 +30,14 @@ namespace mxattn {
 namespace {
 
 constexpr int kQuantThreads = 256;
-constexpr int kUnroll = 4;
+#ifndef MXATTN_QUANT_UNROLL
+#define MXATTN_QUANT_UNROLL 8
+#endif
+#ifndef MXATTN_QUANT_CTAS_PER_SM
+#define MXATTN_QUANT_CTAS_PER_SM 8
+#endif
+constexpr int kUnroll = MXATTN_QUANT_UNROLL;             // 16-byte loads in flight per lane
+constexpr int kCtasPerSm = MXATTN_QUANT_CTAS_PER_SM;     // grid of the grid-stride quantizer
 
 // One 32-element block spread over a quad of lanes (8 elements each).
 // Returns the packed codes of this lane's 8 elements; `e_out` gets the block exponent.
@@ -56,39 +63,23 @@ __device__ __forceinline__ uint32_t quantize_quad(uint4 raw, int uos, int& e_out
     return pack_e2m1x8(f);
 }
 
-// Regrouped scale offset of (row r of a [*, N] operand, block k): per 128-row
-// group, row m sits at byte (m%32)*16 + (m/32)*4 + k.
-__device__ __forceinline__ int64_t regrouped_sf_offset(int64_t bh, int64_t groups, int r, int k) {
-    const int m = r & 127;
-    return (bh * groups + (r >> 7)) * 512 + (m & 31) * 16 + (m >> 5) * 4 + k;
-}
-
 struct RowsArgs {
     const uint16_t* x[2];
     uint8_t* codes[2];
     uint8_t* scales[2];
 };
 
-// Row quantization of up to two tensors (blockIdx.y selects one).
-//   n_chunks: 16-byte chunks per tensor (rows * cols / 8).
-//   regroup == 0: scales are row-major [rows, cols/32].
-//   regroup == 1: rows are (bh, r) with r < N; scales go to the regrouped
-//     layout (cols in {64, 128}) and the scale bytes of the padding rows
-//     r in [N, G*128) are zeroed.
-__global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(RowsArgs a, int64_t n_chunks, int cols,
-                                                                      int uos, int regroup, int N, int groups,
-                                                                      int64_t BH, uint32_t* status) {
-    const uint16_t* __restrict__ x = a.x[blockIdx.y];
-    uint32_t* __restrict__ codes = reinterpret_cast<uint32_t*>(a.codes[blockIdx.y]);
-    uint8_t* __restrict__ scales = a.scales[blockIdx.y];
-    if (status != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status = 0u;
-
+// Row quantization with row-major scales [rows, cols/32] (the standalone op):
+// grid-stride over 16-byte chunks, kUnroll loads in flight per lane.
+__global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(RowsArgs a, int64_t n_chunks, int cols, int uos,
+                                                                      uint32_t* status) {
+    const uint16_t* __restrict__ x = a.x[0];
+    uint32_t* __restrict__ codes = reinterpret_cast<uint32_t*>(a.codes[0]);
+    uint8_t* __restrict__ scales = a.scales[0];
+    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x) >> 5;
     const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * kQuantThreads) >> 5;
-    const int chunk_shift = (cols == 64) ? 3 : 4;  // log2(chunks per row) in regrouped mode
-    const int blocks_per_row = cols >> 5;
-
     for (int64_t base = warp * (32 * kUnroll); base < n_chunks; base += n_warps * (32 * kUnroll)) {
         uint4 raw[kUnroll];
 #pragma unroll
@@ -103,56 +94,86 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(RowsArgs a
             const uint32_t packed = quantize_quad(raw[u], uos, e);
             if (i < n_chunks) {
                 codes[i] = packed;
-                if ((lane & 3) == 0) {
-                    const int64_t blk = i >> 2;
-                    if (!regroup) {
-                        scales[blk] = static_cast<uint8_t>(e + 127);
-                    } else {
-                        const int64_t row = i >> chunk_shift;
-                        const int k = static_cast<int>(blk % blocks_per_row);
-                        const int64_t bh = row / N;
-                        const int r = static_cast<int>(row - bh * N);
-                        scales[regrouped_sf_offset(bh, groups, r, k)] = static_cast<uint8_t>(e + 127);
-                    }
-                }
+                if ((lane & 3) == 0) scales[i >> 2] = static_cast<uint8_t>(e + 127);
             }
-        }
-    }
-    if (regroup) {
-        // zero the scale bytes of padding rows so the tensor core never reads stale bytes
-        const int pad_rows = groups * 128 - N;
-        const int64_t n_pad = BH * pad_rows * blocks_per_row;
-        const int64_t tid = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
-        for (int64_t t = tid; t < n_pad; t += static_cast<int64_t>(gridDim.x) * kQuantThreads) {
-            const int k = static_cast<int>(t % blocks_per_row);
-            const int64_t pr = t / blocks_per_row;
-            const int64_t bh = pr / pad_rows;
-            const int r = N + static_cast<int>(pr - bh * pad_rows);
-            scales[regrouped_sf_offset(bh, groups, r, k)] = 0;
         }
     }
 }
 
-// V^T quantization: grid (G token groups of 128, BH).  Shared tile [128][D] bf16.
+// Forward's Q/K quantization: one CTA per (128-row group, bh, tensor).  Rows
+// past N are zeros; the group's 512 scale bytes are assembled in shared memory
+// in the regrouped order and written out contiguously.
 template <int D>
-__global__ void __launch_bounds__(kQuantThreads) quantize_vt_kernel(const uint16_t* __restrict__ v, int N, int npad,
-                                                                    int uos, int regroup, int groups,
-                                                                    uint8_t* __restrict__ codes_t,
-                                                                    uint8_t* __restrict__ scales_t) {
+__global__ void __launch_bounds__(kQuantThreads) quantize_rows_grouped_kernel(RowsArgs a, int N, int groups, int uos,
+                                                                              uint32_t* status) {
+    constexpr int kChunksPerRow = D / 8;                          // 16-byte chunks per row
+    constexpr int kPerThread = 128 * kChunksPerRow / kQuantThreads;
+    __shared__ __align__(16) uint8_t sf[512];
+    const uint16_t* __restrict__ x = blockIdx.z ? a.x[1] : a.x[0];
+    uint32_t* __restrict__ codes = reinterpret_cast<uint32_t*>(blockIdx.z ? a.codes[1] : a.codes[0]);
+    uint8_t* __restrict__ scales = blockIdx.z ? a.scales[1] : a.scales[0];
+    const int g = blockIdx.x;
+    const int64_t bh = blockIdx.y;
+    if (status != nullptr && g == 0 && bh == 0 && blockIdx.z == 0 && threadIdx.x == 0) *status = 0u;
+    reinterpret_cast<uint32_t*>(sf)[threadIdx.x & 127] = 0u;
+    const int64_t row0 = bh * N + static_cast<int64_t>(g) * 128;  // global row of the group's first row
+    const int rows_valid = min(128, N - g * 128);
+    uint4 raw[kPerThread];
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+        const int c = threadIdx.x + u * kQuantThreads;
+        const int m = c / kChunksPerRow;
+        raw[u] = (m < rows_valid) ? __ldcs(reinterpret_cast<const uint4*>(x + (row0 + m) * D) + (c % kChunksPerRow))
+                                  : make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();  // sf cleared
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+        const int c = threadIdx.x + u * kQuantThreads;
+        const int m = c / kChunksPerRow;
+        int e;
+        const uint32_t packed = quantize_quad(raw[u], uos, e);
+        if (m < rows_valid) codes[(row0 + m) * (D / 8) + (c % kChunksPerRow)] = packed;
+        if ((threadIdx.x & 3) == 0) {
+            const int k = (c % kChunksPerRow) / 4;
+            sf[(m & 31) * 16 + (m >> 5) * 4 + k] = static_cast<uint8_t>(e + 127);  // zero rows give e = -127
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < 32)
+        reinterpret_cast<uint4*>(scales + (bh * groups + g) * 512)[threadIdx.x] =
+            reinterpret_cast<const uint4*>(sf)[threadIdx.x];
+}
+
+// V^T quantization: grid (G token groups of 128, BH), D threads.  The CTA stages
+// 128 tokens x D channels (bf16) in shared memory; thread `ch` then quantizes
+// the four 32-token blocks of its channel and writes 64 contiguous code bytes.
+template <int D>
+__global__ void __launch_bounds__(D) quantize_vt_kernel(const uint16_t* __restrict__ v, int N, int npad, int uos,
+                                                        int regroup, int groups, uint8_t* __restrict__ codes_t,
+                                                        uint8_t* __restrict__ scales_t) {
     __shared__ __align__(16) uint16_t tile[128 * D];
     const int g = blockIdx.x;
     const int64_t bh = blockIdx.y;
     const int t0 = g * 128;
+    const int ch = threadIdx.x;
     constexpr int kChunksPerRow = D / 8;
-    for (int c = threadIdx.x; c < 128 * kChunksPerRow; c += kQuantThreads) {
-        const int t = c / kChunksPerRow, q = c % kChunksPerRow;
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (t0 + t < N) val = __ldcs(reinterpret_cast<const uint4*>(v + ((bh * N + t0 + t) * D)) + q);
-        reinterpret_cast<uint4*>(tile)[c] = val;
+    constexpr int kPerThread = 128 * kChunksPerRow / D;  // 16 loads of 16 bytes in flight
+    uint4 val[kPerThread];
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+        const int c = ch + u * D;
+        const int t = c / kChunksPerRow;
+        val[u] = (t0 + t < N) ? __ldcs(reinterpret_cast<const uint4*>(v + (bh * N + t0 + t) * D) + (c % kChunksPerRow))
+                              : make_uint4(0, 0, 0, 0);
     }
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) reinterpret_cast<uint4*>(tile)[ch + u * D] = val[u];
     __syncthreads();
-    for (int item = threadIdx.x; item < D * 4; item += kQuantThreads) {
-        const int ch = item % D, k = item / D;
+    uint32_t sfword = 0;
+    uint8_t* rowp = codes_t + (bh * D + ch) * static_cast<int64_t>(npad / 2);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
         uint32_t amax = 0;
         uint32_t raw[32];
 #pragma unroll
@@ -171,24 +192,20 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_vt_kernel(const uint16
             words[w] = pack_e2m1x8(f);
         }
         const int tb = t0 + 32 * k;  // first token of the block
-        if (tb < npad) {
-            uint8_t* dst = codes_t + (bh * D + ch) * static_cast<int64_t>(npad / 2) + tb / 2;
-            *reinterpret_cast<uint4*>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
-        }
-        const uint8_t sbyte = static_cast<uint8_t>(e + 127);
-        if (!regroup) {
-            if (tb < npad) scales_t[(bh * D + ch) * static_cast<int64_t>(npad / 32) + tb / 32] = sbyte;
-        } else {
-            // group g of 128 tokens; channel ch plays the role of the row
-            scales_t[(bh * groups + g) * 512 + (ch & 31) * 16 + (ch >> 5) * 4 + k] = sbyte;
-        }
+        if (tb < npad) *reinterpret_cast<uint4*>(rowp + tb / 2) = make_uint4(words[0], words[1], words[2], words[3]);
+        const uint32_t sbyte = static_cast<uint32_t>(e + 127);
+        sfword |= sbyte << (8 * k);
+        if (!regroup && tb < npad) scales_t[(bh * D + ch) * static_cast<int64_t>(npad / 32) + tb / 32] = sbyte;
     }
-    if (regroup && D < 128) {
-        // channel rows D..127 of the group: scale 2^0, so the extra ones-row the
-        // attention kernel appends to V^T (row D) is read with unit scale
-        for (int idx = threadIdx.x; idx < (128 - D) * 4; idx += kQuantThreads) {
-            const int ch = D + idx / 4, k = idx % 4;
-            scales_t[(bh * groups + g) * 512 + (ch & 31) * 16 + (ch >> 5) * 4 + k] = 127;
+    if (regroup) {
+        // group g of 128 tokens; channel ch plays the role of the row
+        uint8_t* grp = scales_t + (bh * groups + g) * 512;
+        *reinterpret_cast<uint32_t*>(grp + (ch & 31) * 16 + (ch >> 5) * 4) = sfword;
+        if (D < 128) {
+            // channel rows D..127 of the group: scale 2^0, so the extra ones-row the
+            // attention kernel appends to V^T (row D) is read with unit scale
+            const int c2 = ch + D;
+            *reinterpret_cast<uint32_t*>(grp + (c2 & 31) * 16 + (c2 >> 5) * 4) = 0x7F7F7F7Fu;
         }
     }
 }
@@ -235,7 +252,7 @@ int grid_for(int64_t work_items, int per_block) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t want = (work_items + per_block - 1) / per_block;
-    const int64_t cap = static_cast<int64_t>(sms) * 8;  // 8 resident CTAs of 256 threads per SM
+    const int64_t cap = static_cast<int64_t>(sms) * kCtasPerSm;
     return static_cast<int>(want < 1 ? 1 : (want < cap ? want : cap));
 }
 
@@ -250,9 +267,17 @@ cudaError_t launch_quantize_rows(const void* const* x, uint8_t* const* codes, ui
         a.codes[t] = codes[t];
         a.scales[t] = scales[t];
     }
+    if (regroup) {
+        dim3 grid(groups, static_cast<unsigned>(BH), ntensors);
+        if (cols == 128)
+            quantize_rows_grouped_kernel<128><<<grid, kQuantThreads, 0, stream>>>(a, N, groups, uos, status);
+        else
+            quantize_rows_grouped_kernel<64><<<grid, kQuantThreads, 0, stream>>>(a, N, groups, uos, status);
+        return cudaGetLastError();
+    }
     const int64_t n_chunks = rows * cols / 8;
     dim3 grid(grid_for(n_chunks / kUnroll, kQuantThreads), ntensors);
-    quantize_rows_kernel<<<grid, kQuantThreads, 0, stream>>>(a, n_chunks, cols, uos, regroup, N, groups, BH, status);
+    quantize_rows_kernel<<<grid, kQuantThreads, 0, stream>>>(a, n_chunks, cols, uos, status);
     return cudaGetLastError();
 }
 
@@ -261,11 +286,11 @@ cudaError_t launch_quantize_vt(const void* v, int64_t BH, int N, int d, int uos,
     const int npad = (N + 31) / 32 * 32;
     dim3 grid(groups, static_cast<unsigned>(BH));
     if (d == 128)
-        quantize_vt_kernel<128><<<grid, kQuantThreads, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, uos,
-                                                                    regroup, groups, codes_t, scales_t);
+        quantize_vt_kernel<128><<<grid, 128, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, uos, regroup,
+                                                           groups, codes_t, scales_t);
     else
-        quantize_vt_kernel<64><<<grid, kQuantThreads, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, uos,
-                                                                   regroup, groups, codes_t, scales_t);
+        quantize_vt_kernel<64><<<grid, 64, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, uos, regroup, groups,
+                                                         codes_t, scales_t);
     return cudaGetLastError();
 }
 
