@@ -227,6 +227,23 @@ def quantize_sweep_point(torch, mx, peaks, peak_kind, log2n=30, iters=10):
     return out
 
 
+# Exponentials per S element in mxattn_fwd_kernel: three of every four pairs on
+# the MUFU (ex2.approx), one on the FMA pipe; plus one per 32-column block.
+MUFU_EX2_PER_ELEMENT = 0.75 + 1.0 / 32
+
+
+def mufu_roofline(w, attn_ms, clocks, sms=148, ex2_per_clk_per_sm=16):
+    """The unit that actually bounds the attention kernel: ex2.approx issue on the
+    MUFU (16 per clock per SM, measured), at the SM clock seen during the run."""
+    mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    elements = float(w.B * w.H) * w.N * w.N
+    achieved = elements * MUFU_EX2_PER_ELEMENT / (attn_ms / 1e3)
+    peak = sms * ex2_per_clk_per_sm * mhz * 1e6
+    return {"bound": "mufu", "unit": "ex2/s", "achieved": achieved, "peak": peak, "frac": achieved / peak,
+            "ex2_per_element": MUFU_EX2_PER_ELEMENT, "sm_mhz": mhz,
+            "s_elements_per_clk_per_sm": elements / (attn_ms / 1e3) / (sms * mhz * 1e6)}
+
+
 def max_over_ranks(values, dist=None, device="cpu"):
     """Element-wise maximum of per-rank timings (the slowest rank counts); identity without a process group."""
     import torch
@@ -321,6 +338,24 @@ def run_gpu(args, rank, world, local_rank):
     if rank == 0 and not args.quick and not args.no_quantize_sweep:
         quant = quantize_sweep_point(torch, mx, peaks, peak_kind)
 
+    # The same attention step with the OCP rule and no PNQ (the comparator the
+    # method is measured against): the cost of UOS + PNQ relative to it.
+    overhead = None
+    if not args.quick:
+        mx.mxattn_prepare(q, k, v, "ocp", ws)
+        for _ in range(2):
+            mx.mxattn_attend(ws, B, H, N, d, w.kv_tile, False, "ocp", 0.0, out)
+        torch.cuda.synchronize()
+        o0, o1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        o0.record(stream)
+        for _ in range(5):
+            mx.mxattn_attend(ws, B, H, N, d, w.kv_tile, False, "ocp", 0.0, out)
+        o1.record(stream)
+        torch.cuda.synchronize()
+        ocp_ms = max_over_ranks([o0.elapsed_time(o1) / 5], dist, "cuda")[0]
+        overhead = {"ocp_no_pnq_attn_ms": ocp_ms, "uos_pnq_attn_ms": attn_avg_ms,
+                    "uos_pnq_over_ocp": attn_avg_ms / ocp_ms - 1.0}
+
     if rank == 0:
         attn_tflops = w.flops / (attn_avg_ms / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
@@ -343,6 +378,8 @@ def run_gpu(args, rank, world, local_rank):
                 "value": world * w.flops / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": 3 * B * H * N * d * 2, "d2h_bytes_per_step": B * H * N * d * 4,
                 "ms_per_step": e2e_ms, "api": "attention_from_host -> mxattn_forward"},
+            "mufu_roofline": mufu_roofline(w, attn_avg_ms, clocks),
+            "uos_pnq_overhead": overhead,
             "gpu_launches": 3 * args.steps,
             "clocks": clocks,
             "quantize_sweep": quant,

@@ -183,6 +183,25 @@ mxattn_status mxattn_forward_noalloc(const void* Q, const void* K, const void* V
  */
 mxattn_status mxattn_workspace_status(const void* workspace, mxattn_stream_t stream);
 
+/*
+ * Failure-detection self-test of the bounded wait that every mbarrier wait in
+ * the attention kernel goes through (this library's own safeguard; the paper
+ * has no counterpart).  Launches one warp on `stream` that waits on a shared
+ * memory mbarrier for phase 0 with a limit of `timeout_us` microseconds
+ * (1 .. 1,000,000).  If `arrive` is non-zero the barrier's single arrival is
+ * made first and the wait completes at once; otherwise nobody arrives and the
+ * wait gives up at its limit, raising the kernel's abort flag.  Nothing
+ * faults: the kernel returns either way and the context stays usable.
+ *   out: device u32[3], 4-byte aligned, written by the kernel:
+ *        out[0] = 0 (completed) or MXATTN_ERR_TIMEOUT (gave up),
+ *        out[1] = microseconds the warp spent waiting,
+ *        out[2] = bit 0 abort flag raised, bit 1 wait left without completion.
+ * Returns MXATTN_ERR_INVALID (null/misaligned out, timeout out of range) or
+ * MXATTN_ERR_CUDA (launch failed); otherwise MXATTN_OK (asynchronous: read
+ * `out` after synchronizing `stream`).
+ */
+mxattn_status mxattn_wait_selftest(int arrive, unsigned timeout_us, unsigned* out, mxattn_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* mxattn_status_string(mxattn_status status);
 

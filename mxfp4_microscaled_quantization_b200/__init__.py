@@ -17,6 +17,7 @@ from .mxattn import (  # noqa: F401
     mxattn_quantize,
     mxattn_quantize_vt,
     mxattn_status_string,
+    mxattn_wait_selftest,
     mxattn_workspace_size,
     mxattn_workspace_status,
     new_workspace,

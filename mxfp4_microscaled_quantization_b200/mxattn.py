@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.mxattn_forward_noalloc.restype = i32
         L.mxattn_workspace_status.argtypes = [P, P]
         L.mxattn_workspace_status.restype = i32
+        L.mxattn_wait_selftest.argtypes = [i32, ctypes.c_uint, P, P]
+        L.mxattn_wait_selftest.restype = i32
         _lib = L
     return _lib
 
@@ -233,6 +235,15 @@ def mxattn_forward_noalloc(q, k, v, kv_tile=128, pnq=True, rule="uos", softmax_s
 def mxattn_workspace_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronize and return the status word of the last forward on `workspace` (0 = ok)."""
     return int(lib().mxattn_workspace_status(_cuda(workspace, "workspace"), _stream(stream)))
+
+
+def mxattn_wait_selftest(arrive: bool, timeout_us: int, out: torch.Tensor, stream=None) -> None:
+    """Launch the bounded-wait self-test; `out` is a device int32[3] tensor that
+    holds (status, microseconds waited, flags) once the stream is synchronized."""
+    if out.dtype != torch.int32 or out.numel() < 3 or not out.is_contiguous():
+        raise MxattnError(1, "out must be a contiguous int32 tensor with 3 elements")
+    _check(lib().mxattn_wait_selftest(int(bool(arrive)), int(timeout_us), _cuda(out, "out"), _stream(stream)),
+           "mxattn_wait_selftest")
 
 
 def mxattn_status_string(status: int) -> str:
