@@ -237,37 +237,49 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
     // named barrier after which the MMA warp frees TMEM.
     if (warp >= 4 * NT) {
         warpgroup_regs_dec<C::kRoleRegs>();
+        // The producer and the MMA issuer run their loops with the whole warp,
+        // so the loop state stays warp-uniform; one elected lane (fixed for
+        // the kernel) issues every copy and tcgen05 instruction.
+        const bool leader = elect_one_sync();
+        auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag, p.status, kTimeoutCode,
+                                                             kTimeoutNs, kRoleWaitHintNs));
+        };
         if (warp == C::kProducerWarp) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
             int k_issued = 0, v_issued = 0;
-            mbar_arrive_expect_tx(bar_q, NT * (C::kQBytes + C::kSfBytes));
-            for (int t = 0; t < NT; ++t) {
-                const int g = 2 * qp + t;  // 128-row group of tile t (may lie past N: zero-filled)
-                tma_load_3d(sQ + t * C::kQBytes, &tmQ, bar_q, 0, g * 128, bh);
-                const int gs = g < p.groups ? g : p.groups - 1;  // keep the scale copy inside the buffer
-                bulk_load(sQsf + t * 512, p.q_sf + (static_cast<size_t>(bh) * p.groups + gs) * 512, 512, bar_q);
+            if (leader) {
+                mbar_arrive_expect_tx(bar_q, NT * (C::kQBytes + C::kSfBytes));
+                for (int t = 0; t < NT; ++t) {
+                    const int g = 2 * qp + t;  // 128-row group of tile t (may lie past N: zero-filled)
+                    tma_load_3d(sQ + t * C::kQBytes, &tmQ, bar_q, 0, g * 128, bh);
+                    const int gs = g < p.groups ? g : p.groups - 1;  // keep the scale copy inside the buffer
+                    bulk_load(sQsf + t * 512, p.q_sf + (static_cast<size_t>(bh) * p.groups + gs) * 512, 512, bar_q);
+                }
             }
+            __syncwarp();
             for (int j = 0; j < nkv; ++j) {
                 const int s = j % S;
                 const uint32_t n = j / S;
                 const size_t grp = static_cast<size_t>(bh) * p.groups + (j * T) / 128;
-                if (j >= S && !mbar_wait_bounded(bar_k_empty + s, (n - 1) & 1, abort_flag, p.status, kTimeoutCode,
-                                                 kTimeoutNs, kRoleWaitHintNs))
-                    break;
-                mbar_arrive_expect_tx(bar_k_full + s, C::kKBytes + C::kSfBytes);
-                tma_load_3d(sK + s * C::kKBytes, &tmK, bar_k_full + s, 0, j * T, bh);
-                bulk_load(sKsf + s * 512, p.k_sf + grp * 512, 512, bar_k_full + s);
+                if (j >= S && !wait(bar_k_empty + s, (n - 1) & 1)) break;
+                if (leader) {
+                    mbar_arrive_expect_tx(bar_k_full + s, C::kKBytes + C::kSfBytes);
+                    tma_load_3d(sK + s * C::kKBytes, &tmK, bar_k_full + s, 0, j * T, bh);
+                    bulk_load(sKsf + s * 512, p.k_sf + grp * 512, 512, bar_k_full + s);
+                }
+                __syncwarp();
                 k_issued = j + 1;
-                if (j >= S && !mbar_wait_bounded(bar_v_empty + s, (n - 1) & 1, abort_flag, p.status, kTimeoutCode,
-                                                 kTimeoutNs, kRoleWaitHintNs))
-                    break;
-                mbar_arrive_expect_tx(bar_v_full + s, C::kVLoadBytes + C::kSfBytes);
-                tma_load_3d(sV + s * C::kVStride, &tmV, bar_v_full + s, j * (T / 2), 0, bh);
-                bulk_load(sVsf + s * 512, p.v_sf + grp * 512, 512, bar_v_full + s);
+                if (j >= S && !wait(bar_v_empty + s, (n - 1) & 1)) break;
+                if (leader) {
+                    mbar_arrive_expect_tx(bar_v_full + s, C::kVLoadBytes + C::kSfBytes);
+                    tma_load_3d(sV + s * C::kVStride, &tmV, bar_v_full + s, j * (T / 2), 0, bh);
+                    bulk_load(sVsf + s * 512, p.v_sf + grp * 512, 512, bar_v_full + s);
+                }
+                __syncwarp();
                 v_issued = j + 1;
             }
-            // Drain: every copy this thread issued must land before the CTA exits.
+            // Drain: every copy the leader issued must land before the CTA exits.
             // On the normal path these phases completed long ago and the waits return at once.
             int dummy = 0;
             volatile int* no_abort = &dummy;
@@ -277,33 +289,37 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                 mbar_wait_bounded(bar_k_full + j % S, (j / S) & 1, no_abort, p.status, kTimeoutCode, kTimeoutNs);
             for (int j = v_issued - S < 0 ? 0 : v_issued - S; j < v_issued; ++j)
                 mbar_wait_bounded(bar_v_full + j % S, (j / S) & 1, no_abort, p.status, kTimeoutCode, kTimeoutNs);
-        }
+            __syncwarp();
     } else if (warp == C::kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
             const uint32_t t_s = tbase + C::kColS;
-            auto wait = [&](uint64_t* bar, uint32_t parity) {
-                return mbar_wait_bounded(bar, parity, abort_flag, p.status, kTimeoutCode, kTimeoutNs, kRoleWaitHintNs);
-            };
+            // Shared-memory descriptors of the first buffer of each operand; a buffer
+            // b bytes further on is the descriptor plus b >> 4 (start-address field).
+            const uint64_t qdesc0 = smem_desc(smem_u32(sQ), 16, C::kQKSbo, C::kQKLayout);
+            const uint64_t kdesc0 = smem_desc(smem_u32(sK), 16, C::kQKSbo, C::kQKLayout);
+            const uint64_t pdesc0 = smem_desc(smem_u32(sP), 16, C::kPVSbo, C::kPVLayout);
+            const uint64_t vdesc0 = smem_desc(smem_u32(sV), 16, C::kPVSbo, C::kPVLayout);
+            const uint64_t ksf0 = sf_desc(sKsf), vsf0 = sf_desc(sVsf), psf0 = sf_desc(sPsf);
             // S_t(j) = Q_t K(j)^T into the shared S buffer.  Tile A's issue also
             // waits for K(j) and copies its scales; tile B reuses both.
             auto issue_s = [&](int t, int j) -> bool {
                 const int s = j % S;
                 const uint32_t n = j / S;
-                if (t == 0) {
-                    if (!wait(bar_k_full + s, n & 1)) return false;
-                    tc_fence_after_sync();
-                    tc_cp_sf(tbase + C::kColKsf + 4 * s, sf_desc(sKsf + s * 512));
-                }
-                const uint64_t qdesc = smem_desc(smem_u32(sQ + t * C::kQBytes), 16, C::kQKSbo, C::kQKLayout);
-                const uint64_t kdesc = smem_desc(smem_u32(sK + s * C::kKBytes), 16, C::kQKSbo, C::kQKLayout);
+                if (t == 0 && !wait(bar_k_full + s, n & 1)) return false;
+                tc_fence_after_sync();  // after the K wait, or after the wait for the S buffer to be read
+                const uint64_t qdesc = qdesc0 + static_cast<uint32_t>(t * (C::kQBytes >> 4));
+                const uint64_t kdesc = kdesc0 + static_cast<uint32_t>(s * (C::kKBytes >> 4));
                 const uint32_t ksf = tbase + C::kColKsf + 4 * s + ((T == 64) ? 2 * (j & 1) : 0);
+                if (leader) {
+                    if (t == 0) tc_cp_sf(tbase + C::kColKsf + 4 * s, ksf0 + static_cast<uint32_t>(s * (512 >> 4)));
 #pragma unroll
-                for (int kk = 0; kk < D / 64; ++kk)
-                    tc_mma_mxf4(t_s, qdesc + 2 * kk, kdesc + 2 * kk, mxf4_idesc(T, 2 * kk, 2 * kk),
-                                tbase + C::kColQsf + 4 * t, ksf, kk > 0 ? 1u : 0u);
-                tc_commit(bar_s_full + t);
-                if (t == NT - 1) tc_commit(bar_k_empty + s);
+                    for (int kk = 0; kk < D / 64; ++kk)
+                        tc_mma_mxf4(t_s, qdesc + 2 * kk, kdesc + 2 * kk, mxf4_idesc(T, 2 * kk, 2 * kk),
+                                    tbase + C::kColQsf + 4 * t, ksf, kk > 0 ? 1u : 0u);
+                    tc_commit(bar_s_full + t);
+                    if (t == NT - 1) tc_commit(bar_k_empty + s);
+                }
+                __syncwarp();
                 return true;
             };
             // O_t += P_t V(j).  Tile A's issue waits for V(j) and copies its scales.
@@ -313,27 +329,33 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                 if (!wait(bar_p_full + t, j & 1)) return false;
                 if (t == 0 && !wait(bar_v_full + s, n & 1)) return false;
                 tc_fence_after_sync();
-                tc_cp_sf(tbase + C::kColPsf + 4 * t, sf_desc(sPsf + t * 512));
-                if (t == 0) tc_cp_sf(tbase + C::kColVsf + 8 * s, sf_desc(sVsf + s * 512));
-                const uint64_t pdesc = smem_desc(smem_u32(sP + t * C::kPBytes), 16, C::kPVSbo, C::kPVLayout);
-                const uint64_t vdesc = smem_desc(smem_u32(sV + s * C::kVStride), 16, C::kPVSbo, C::kPVLayout);
+                const uint64_t pdesc = pdesc0 + static_cast<uint32_t>(t * (C::kPBytes >> 4));
+                const uint64_t vdesc = vdesc0 + static_cast<uint32_t>(s * (C::kVStride >> 4));
+                if (leader) {
+                    tc_cp_sf(tbase + C::kColPsf + 4 * t, psf0 + static_cast<uint32_t>(t * (512 >> 4)));
+                    if (t == 0) tc_cp_sf(tbase + C::kColVsf + 8 * s, vsf0 + static_cast<uint32_t>(s * (512 >> 4)));
 #pragma unroll
-                for (int kk = 0; kk < T / 64; ++kk) {
-                    const uint32_t sfb_id = (T == 64) ? 2u * (j & 1) : 2u * kk;
-                    tc_mma_mxf4(tbase + C::kColO + t * C::kOCols, pdesc + 2 * kk, vdesc + 2 * kk,
-                                mxf4_idesc(D + 16, 2 * kk, sfb_id), tbase + C::kColPsf + 4 * t,
-                                tbase + C::kColVsf + 8 * s, (j > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < T / 64; ++kk) {
+                        const uint32_t sfb_id = (T == 64) ? 2u * (j & 1) : 2u * kk;
+                        tc_mma_mxf4(tbase + C::kColO + t * C::kOCols, pdesc + 2 * kk, vdesc + 2 * kk,
+                                    mxf4_idesc(D + 16, 2 * kk, sfb_id), tbase + C::kColPsf + 4 * t,
+                                    tbase + C::kColVsf + 8 * s, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc_commit(bar_o_done + t);
+                    if (t == NT - 1) tc_commit(bar_v_empty + s);
                 }
-                tc_commit(bar_o_done + t);
-                if (t == NT - 1) tc_commit(bar_v_empty + s);
+                __syncwarp();
                 return true;
             };
             bool ok = wait(bar_q, 0);
             if (ok) {
                 tc_fence_after_sync();
-                for (int t = 0; t < NT; ++t) tc_cp_sf(tbase + C::kColQsf + 4 * t, sf_desc(sQsf + t * 512));
-                if (D == 128)
-                    for (int s = 0; s < S; ++s) tc_cp_sf(tbase + C::kColVsf + 8 * s + 4, sf_desc(sVsfConst));
+                if (leader) {
+                    for (int t = 0; t < NT; ++t) tc_cp_sf(tbase + C::kColQsf + 4 * t, sf_desc(sQsf + t * 512));
+                    if (D == 128)
+                        for (int s = 0; s < S; ++s) tc_cp_sf(tbase + C::kColVsf + 8 * s + 4, sf_desc(sVsfConst));
+                }
+                __syncwarp();
             }
             // Order: S_A(0); S_B(0) after A loaded; S_A(1) after B loaded; then per tile j:
             // PV_A(j), S_B(j+1) (after A loaded S_A(j+1)), PV_B(j), S_A(j+2) (after B loaded S_B(j+1)).
@@ -346,11 +368,12 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                 if (!issue_pv(1, j)) break;
                 if (j + 2 < nkv && !(wait(bar_s_loaded + 1, (j + 1) & 1) && issue_s(0, j + 2))) break;
             }
-            // Drain: wait for every MMA / copy this thread issued before TMEM is freed.
-            tc_commit(bar_drain);
+            // Drain: wait for every MMA / copy the leader issued before TMEM is freed.
+            if (leader) tc_commit(bar_drain);
+            __syncwarp();
             int dummy = 0;
             mbar_wait_bounded(bar_drain, 0, &dummy, p.status, kTimeoutCode, kTimeoutNs);
-        }
+            __syncwarp();
     }
     tc_fence_before_sync();
     named_barrier_sync(1, C::kThreads);
