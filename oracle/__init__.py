@@ -27,6 +27,8 @@ _SRC = os.path.join(_HERE, "oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
 RULES = {"ocp": 0, "uos": 1, "none": 2}
+RULE_QMAX = 3  # boundary rule with a caller-chosen Qmax in (4, 8)
+UOS_QMAX = 7.25
 
 
 def build(force: bool = False) -> str:
@@ -52,6 +54,12 @@ def lib():
         i64 = ctypes.c_int64
         L.oracle_e2m1_encode_batch.argtypes = [P, i64, P]
         L.oracle_scale_exponent_batch.argtypes = [P, i64, ctypes.c_int, P]
+        L.oracle_scale_exponent_q_batch.argtypes = [P, i64, ctypes.c_int, ctypes.c_double, P]
+        L.oracle_quantize_rows_q.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_double, P, P]
+        L.oracle_quantize_cols_q.argtypes = [P, i64, i64, i64, ctypes.c_int, ctypes.c_double, P, P]
+        L.oracle_attention_head_q.argtypes = [P, P, P, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                              ctypes.c_int, ctypes.c_double, P, i64, P, ctypes.c_int]
+        L.oracle_attention_head_q.restype = ctypes.c_int
         L.oracle_quantize_rows.argtypes = [P, i64, i64, ctypes.c_int, P, P]
         L.oracle_quantize_cols.argtypes = [P, i64, i64, i64, ctypes.c_int, P, P]
         L.oracle_dequantize_rows.argtypes = [P, P, i64, i64, P]
@@ -70,8 +78,20 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
-def _rule(r) -> int:
-    return RULES[r] if isinstance(r, str) else int(r)
+def _rule(r):
+    """Rule name ("ocp", "uos", "none") or a scale boundary Qmax -> (rule code, Qmax).
+
+    A numeric Qmax in (4, 8) selects the boundary rule "smallest e with
+    amax <= Qmax * 2^e"; Qmax = 8 selects OCP, the limit of that rule as Qmax
+    approaches 8 from below."""
+    if isinstance(r, str):
+        return RULES[r], UOS_QMAX
+    q = float(r)
+    if q == 8.0:
+        return RULES["ocp"], q
+    if not 4.0 < q < 8.0:
+        raise ValueError(f"Qmax must lie in (4, 8], got {q}")
+    return RULE_QMAX, q
 
 
 def max_threads() -> int:
@@ -93,7 +113,8 @@ def e2m1_encode(v) -> np.ndarray:
 def scale_exponent(amax, rule) -> np.ndarray:
     a = np.ascontiguousarray(amax, dtype=np.float64)
     out = np.empty(a.shape, dtype=np.int32)
-    lib().oracle_scale_exponent_batch(_ptr(a), a.size, _rule(rule), _ptr(out))
+    code, q = _rule(rule)
+    lib().oracle_scale_exponent_q_batch(_ptr(a), a.size, code, q, _ptr(out))
     return out
 
 
@@ -105,7 +126,8 @@ def quantize_rows(x_bits: np.ndarray, rule):
     rows = x.size // cols
     codes = np.empty(x.shape[:-1] + (cols // 2,), dtype=np.uint8)
     scales = np.empty(x.shape[:-1] + (cols // 32,), dtype=np.uint8)
-    lib().oracle_quantize_rows(_ptr(x), rows, cols, _rule(rule), _ptr(codes), _ptr(scales))
+    code, q = _rule(rule)
+    lib().oracle_quantize_rows_q(_ptr(x), rows, cols, code, q, _ptr(codes), _ptr(scales))
     return codes, scales
 
 
@@ -118,7 +140,8 @@ def quantize_cols(v_bits: np.ndarray, rule):
     lead = v.shape[:-2]
     codes = np.empty(lead + (d, npad // 2), dtype=np.uint8)
     scales = np.empty(lead + (d, npad // 32), dtype=np.uint8)
-    lib().oracle_quantize_cols(_ptr(v), BH, N, d, _rule(rule), _ptr(codes), _ptr(scales))
+    code, q = _rule(rule)
+    lib().oracle_quantize_cols_q(_ptr(v), BH, N, d, code, q, _ptr(codes), _ptr(scales))
     return codes, scales
 
 
@@ -136,7 +159,9 @@ def attention(Q, K, V, kv_tile, rule="uos", pnq=True, p_rule=None, scale=None, r
     """MXFP4 attention forward on the CPU in fp64.
 
     Q, K, V: bf16 bits [B, H, N, d].  `rule` quantizes Q, K, V (and P unless
-    `p_rule` says otherwise); "none" disables quantization.  `rows`: None for
+    `p_rule` says otherwise); "none" disables quantization; a number is a
+    scale boundary Qmax in (4, 8] (see `_rule`).  A numeric `rule` and a
+    numeric `p_rule` must name the same Qmax.  `rows`: None for
     all rows, else an int array of query rows (the same rows for every head)
     or a list with one array per (b, h).  Returns fp64 [B, H, R, d].
     """
@@ -146,8 +171,11 @@ def attention(Q, K, V, kv_tile, rule="uos", pnq=True, p_rule=None, scale=None, r
     B, H, N, d = Q.shape
     if scale is None or scale <= 0:
         scale = 1.0 / math.sqrt(d)
-    in_rule = _rule(rule)
-    pr = in_rule if p_rule is None else _rule(p_rule)
+    in_rule, q_in = _rule(rule)
+    pr, q_p = (in_rule, q_in) if p_rule is None else _rule(p_rule)
+    qmax = q_in if in_rule == RULE_QMAX else q_p
+    if in_rule == RULE_QMAX and pr == RULE_QMAX and q_in != q_p:
+        raise ValueError("rule and p_rule must name the same Qmax")
     per_head_rows = []
     for bh in range(B * H):
         if rows is None:
@@ -166,9 +194,9 @@ def attention(Q, K, V, kv_tile, rule="uos", pnq=True, p_rule=None, scale=None, r
     ov = out.reshape(B * H, R, d)
     for bh in range(B * H):
         o = np.empty((R, d), dtype=np.float64)
-        st = lib().oracle_attention_head(_ptr(Qf[bh]), _ptr(Kf[bh]), _ptr(Vf[bh]), N, d, kv_tile, in_rule, pr,
-                                         1 if pnq else 0, float(scale), _ptr(per_head_rows[bh]), R, _ptr(o),
-                                         int(nthreads))
+        st = lib().oracle_attention_head_q(_ptr(Qf[bh]), _ptr(Kf[bh]), _ptr(Vf[bh]), N, d, kv_tile, in_rule, pr,
+                                           float(qmax), 1 if pnq else 0, float(scale), _ptr(per_head_rows[bh]), R,
+                                           _ptr(o), int(nthreads))
         if st != 0:
             raise RuntimeError(f"oracle_attention_head failed with status {st}")
         ov[bh] = o

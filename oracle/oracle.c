@@ -17,6 +17,9 @@
  *     with a sign bit, one E8M0 power-of-two scale per block.
  *   - OCP scale rule: e = floor(log2 amax) - 2 (2 = largest E2M1 exponent).
  *   - UOS scale rule: the smallest integer e with amax <= 7.25 * 2^e.
+ *   - the same boundary rule for any Qmax in (4, 8) (the abstract names the
+ *     boundary Qmax; 7.25 is its choice), used to sweep the boundary; OCP is
+ *     the limit Qmax -> 8 from below (reading).
  *   - elements: round to nearest, ties to the even code, saturate at 6.
  *
  * Every loop follows the definitions in the order the method states them;
@@ -34,6 +37,7 @@
 #define ORACLE_RULE_OCP 0
 #define ORACLE_RULE_UOS 1
 #define ORACLE_RULE_NONE 2 /* identity: no quantization at all */
+#define ORACLE_RULE_QMAX 3 /* boundary rule with a caller-chosen Qmax in (4, 8) */
 
 /* E2M1 magnitudes in code order (code bits: sign | exponent(2) | mantissa(1)). */
 static const double kE2M1Magnitude[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
@@ -89,10 +93,12 @@ void oracle_e2m1_encode_batch(const double* v, int64_t n, uint8_t* codes) {
  *   UOS (abstract: data-free boundary Qmax = 7.25): smallest e with
  *       amax <= Qmax * 2^e, so amax / 2^e lies in (Qmax/2, Qmax]; values in
  *       (6, Qmax] then saturate to 6.
+ *   QMAX: the same boundary rule with the caller's Qmax (reading: any
+ *       boundary in (4, 8) is a valid member of the family UOS picks from).
  * Reading for the cases the pages leave open: amax == 0 (or not > 0) gives
  * e = -127; e is clamped to the E8M0 range [-127, 127].
  */
-int oracle_scale_exponent(double amax, int rule) {
+static int scale_exponent(double amax, int rule, double qmax) {
     if (!(amax > 0.0)) return -127;
     int E;
     (void)frexp(amax, &E); /* amax = f * 2^E, f in [0.5, 1)  =>  floor(log2 amax) = E - 1 */
@@ -101,27 +107,34 @@ int oracle_scale_exponent(double amax, int rule) {
     if (rule == ORACLE_RULE_OCP) {
         e = floor_log2 - 2;
     } else {
-        e = floor_log2 - 4; /* Qmax * 2^(floor_log2 - 4) < amax, so the search starts below the answer */
-        while (amax > kUosQmax * ldexp(1.0, e)) e++;
+        double q = (rule == ORACLE_RULE_UOS) ? kUosQmax : qmax;
+        e = floor_log2 - 4; /* q * 2^(floor_log2 - 4) < amax for q < 16: the search starts below the answer */
+        while (amax > q * ldexp(1.0, e)) e++;
     }
     if (e < -127) e = -127;
     if (e > 127) e = 127;
     return e;
 }
 
+int oracle_scale_exponent(double amax, int rule) { return scale_exponent(amax, rule, kUosQmax); }
+
 void oracle_scale_exponent_batch(const double* amax, int64_t n, int rule, int32_t* e) {
-    for (int64_t i = 0; i < n; i++) e[i] = oracle_scale_exponent(amax[i], rule);
+    for (int64_t i = 0; i < n; i++) e[i] = scale_exponent(amax[i], rule, kUosQmax);
+}
+
+void oracle_scale_exponent_q_batch(const double* amax, int64_t n, int rule, double qmax, int32_t* e) {
+    for (int64_t i = 0; i < n; i++) e[i] = scale_exponent(amax[i], rule, qmax);
 }
 
 /* Quantize one block of n values (n <= 32; positions n..31 count as zeros).
  * Returns e; writes n codes.  */
-static int quantize_block(const double* x, int n, int rule, uint8_t* codes) {
+static int quantize_block(const double* x, int n, int rule, double qmax, uint8_t* codes) {
     double amax = 0.0;
     for (int i = 0; i < n; i++) {
         double a = fabs(x[i]);
         if (a > amax) amax = a;
     }
-    int e = oracle_scale_exponent(amax, rule);
+    int e = scale_exponent(amax, rule, qmax);
     for (int i = 0; i < n; i++) codes[i] = oracle_e2m1_encode(ldexp(x[i], -e));
     return e;
 }
@@ -132,19 +145,24 @@ static int quantize_block(const double* x, int n, int rule, uint8_t* codes) {
  * codes: [rows, cols/2] bytes, element 2i in the low nibble, 2i+1 in the high
  * nibble.  scales: [rows, cols/32] E8M0 bytes (e + 127).
  */
-void oracle_quantize_rows(const uint16_t* x, int64_t rows, int64_t cols, int rule,
-                          uint8_t* codes, uint8_t* scales) {
+void oracle_quantize_rows_q(const uint16_t* x, int64_t rows, int64_t cols, int rule, double qmax,
+                            uint8_t* codes, uint8_t* scales) {
     double blk[32];
     uint8_t c[32];
     for (int64_t r = 0; r < rows; r++) {
         for (int64_t b = 0; b < cols / 32; b++) {
             for (int i = 0; i < 32; i++) blk[i] = oracle_bf16_to_double(x[r * cols + b * 32 + i]);
-            int e = quantize_block(blk, 32, rule, c);
+            int e = quantize_block(blk, 32, rule, qmax, c);
             scales[r * (cols / 32) + b] = (uint8_t)(e + 127);
             for (int i = 0; i < 16; i++)
                 codes[r * (cols / 2) + b * 16 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
         }
     }
+}
+
+void oracle_quantize_rows(const uint16_t* x, int64_t rows, int64_t cols, int rule, uint8_t* codes,
+                          uint8_t* scales) {
+    oracle_quantize_rows_q(x, rows, cols, rule, kUosQmax, codes, scales);
 }
 
 /*
@@ -153,8 +171,8 @@ void oracle_quantize_rows(const uint16_t* x, int64_t rows, int64_t cols, int rul
  * v: bf16 bits [BH, N, d].  Output is V transposed: codes [BH, d, Npad/2],
  * scales [BH, d, Npad/32], Npad = ceil(N/32)*32, tokens >= N count as zeros.
  */
-void oracle_quantize_cols(const uint16_t* v, int64_t BH, int64_t N, int64_t d, int rule,
-                          uint8_t* codes, uint8_t* scales) {
+void oracle_quantize_cols_q(const uint16_t* v, int64_t BH, int64_t N, int64_t d, int rule, double qmax,
+                            uint8_t* codes, uint8_t* scales) {
     int64_t npad = (N + 31) / 32 * 32;
     double blk[32];
     uint8_t c[32];
@@ -165,13 +183,18 @@ void oracle_quantize_cols(const uint16_t* v, int64_t BH, int64_t N, int64_t d, i
                     int64_t t = b * 32 + i;
                     blk[i] = (t < N) ? oracle_bf16_to_double(v[(bh * N + t) * d + ch]) : 0.0;
                 }
-                int e = quantize_block(blk, 32, rule, c);
+                int e = quantize_block(blk, 32, rule, qmax, c);
                 scales[(bh * d + ch) * (npad / 32) + b] = (uint8_t)(e + 127);
                 for (int i = 0; i < 16; i++)
                     codes[(bh * d + ch) * (npad / 2) + b * 16 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
             }
         }
     }
+}
+
+void oracle_quantize_cols(const uint16_t* v, int64_t BH, int64_t N, int64_t d, int rule, uint8_t* codes,
+                          uint8_t* scales) {
+    oracle_quantize_cols_q(v, BH, N, d, rule, kUosQmax, codes, scales);
 }
 
 /* Dequantize row-layout codes/scales back to values. */
@@ -213,11 +236,12 @@ void oracle_dequantize_rows(const uint8_t* codes, const uint8_t* scales, int64_t
  *     m = m_new
  *   O_i = o / l
  *
+ * qmax: the boundary of ORACLE_RULE_QMAX (both rules; ignored by the others).
  * rows: indices of the query rows to compute; O: [nrows, d] fp64.
  */
-int oracle_attention_head(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int64_t N, int64_t d,
-                          int64_t kv_tile, int in_rule, int p_rule, int pnq, double scale,
-                          const int64_t* rows, int64_t nrows, double* O, int nthreads) {
+int oracle_attention_head_q(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int64_t N, int64_t d,
+                            int64_t kv_tile, int in_rule, int p_rule, double qmax, int pnq, double scale,
+                            const int64_t* rows, int64_t nrows, double* O, int nthreads) {
     if (N < 1 || d % 32 != 0 || kv_tile % 32 != 0 || kv_tile < 32) return 1;
     int64_t npad = (N + 31) / 32 * 32;
     double* kd = (double*)malloc(sizeof(double) * (size_t)(N * d));
@@ -233,7 +257,7 @@ int oracle_attention_head(const uint16_t* Q, const uint16_t* K, const uint16_t* 
     } else {
         uint8_t* c = (uint8_t*)malloc((size_t)(N * d / 2));
         uint8_t* s = (uint8_t*)malloc((size_t)(N * d / 32));
-        oracle_quantize_rows(K, N, d, in_rule, c, s);
+        oracle_quantize_rows_q(K, N, d, in_rule, qmax, c, s);
         oracle_dequantize_rows(c, s, N, d, kd);
         free(c);
         free(s);
@@ -246,7 +270,7 @@ int oracle_attention_head(const uint16_t* Q, const uint16_t* K, const uint16_t* 
     } else {
         uint8_t* c = (uint8_t*)malloc((size_t)(d * npad / 2));
         uint8_t* s = (uint8_t*)malloc((size_t)(d * npad / 32));
-        oracle_quantize_cols(V, 1, N, d, in_rule, c, s);
+        oracle_quantize_cols_q(V, 1, N, d, in_rule, qmax, c, s);
         oracle_dequantize_rows(c, s, d, npad, vt);
         free(c);
         free(s);
@@ -273,7 +297,7 @@ int oracle_attention_head(const uint16_t* Q, const uint16_t* K, const uint16_t* 
             for (int64_t ch = 0; ch < d; ch++) qd[ch] = oracle_bf16_to_double(Q[i * d + ch]);
         } else {
             uint8_t c[64], sc[4];
-            oracle_quantize_rows(Q + i * d, 1, d, in_rule, c, sc);
+            oracle_quantize_rows_q(Q + i * d, 1, d, in_rule, qmax, c, sc);
             oracle_dequantize_rows(c, sc, 1, d, qd);
         }
         /* s_j */
@@ -303,7 +327,7 @@ int oracle_attention_head(const uint16_t* Q, const uint16_t* K, const uint16_t* 
                 if (p_rule == ORACLE_RULE_NONE) {
                     for (int k = 0; k < 32; k++) q[k] = p[k];
                 } else {
-                    int e = quantize_block(p, 32, p_rule, c);
+                    int e = quantize_block(p, 32, p_rule, qmax, c);
                     for (int k = 0; k < 32; k++) q[k] = ldexp(oracle_e2m1_decode(c[k]), e);
                 }
                 for (int k = 0; k < 32; k++) {
@@ -324,6 +348,13 @@ int oracle_attention_head(const uint16_t* Q, const uint16_t* K, const uint16_t* 
     free(kd);
     free(vt);
     return status;
+}
+
+int oracle_attention_head(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int64_t N, int64_t d,
+                          int64_t kv_tile, int in_rule, int p_rule, int pnq, double scale, const int64_t* rows,
+                          int64_t nrows, double* O, int nthreads) {
+    return oracle_attention_head_q(Q, K, V, N, d, kv_tile, in_rule, p_rule, kUosQmax, pnq, scale, rows, nrows, O,
+                                   nthreads);
 }
 
 int oracle_max_threads(void) {

@@ -147,6 +147,83 @@ def test_uos_clip_error_bound():
     assert np.all(a - deq <= np.ldexp(1.25, e) * (1 + 1e-12))
 
 
+# ----------------------------------------------------------------------------- scale boundary Qmax (sweep of the UOS family)
+
+QMAX_SWEEP = [4.5, 5.0, 6.0, 6.5, 7.0, 7.25, 7.5, 7.75, 7.875]
+
+
+def test_qmax_rule_golden_cases():
+    for q, h, _val, e in _read_golden("qmax_rules.txt"):
+        a = float(wl.bf16_bits_to_f32(np.array([int(h, 16)], dtype=np.uint16))[0])
+        assert oracle.scale_exponent([a], float(q))[0] == int(e), (q, h)
+
+
+@pytest.mark.parametrize("q", QMAX_SWEEP)
+def test_qmax_rule_invariant_and_minimality_all_bf16(q):
+    """Boundary rule: amax / 2^e <= Qmax and amax / 2^(e-1) > Qmax for every
+    positive finite bf16 amax whose exponent is not clamped."""
+    bits, a = _all_positive_finite_bf16()
+    e = oracle.scale_exponent(a, q).astype(np.int64)
+    assert np.all(np.ldexp(a, -e) <= q)
+    free = e > -127
+    assert np.all(np.ldexp(a[free], -(e[free] - 1)) > q)
+
+
+@pytest.mark.parametrize("q", QMAX_SWEEP)
+def test_qmax_minus_ocp_closed_form_on_bits(q):
+    """With amax = mu * 2^k (mu in [1, 2)) and Qmax in (4, 8), the boundary rule
+    gives k - 2 + [mu > Qmax/4]: on bf16 bits, mantissa field > floor((Qmax/4 - 1) * 128)."""
+    bits, a = _all_positive_finite_bf16()
+    normal = (bits >> 7) > 1
+    e_o = oracle.scale_exponent(a, "ocp").astype(np.int64)
+    e_q = oracle.scale_exponent(a, q).astype(np.int64)
+    thresh = int(np.floor((q / 4 - 1) * 128))
+    expect = ((bits & 0x7F) > thresh).astype(np.int64)
+    np.testing.assert_array_equal((e_q - e_o)[normal], expect[normal])
+
+
+def test_qmax_rule_contains_uos_and_tends_to_ocp():
+    """Qmax = 7.25 is the UOS rule; a boundary just below 8 gives the OCP exponent
+    for every bf16 maximum (mu < 2 <= Qmax/4 never holds, and mu * 2^k <=
+    Qmax * 2^(k-3) would need mu < 1), and Qmax = 8 names OCP itself."""
+    bits, a = _all_positive_finite_bf16()
+    np.testing.assert_array_equal(oracle.scale_exponent(a, 7.25), oracle.scale_exponent(a, "uos"))
+    np.testing.assert_array_equal(oracle.scale_exponent(a, 8.0), oracle.scale_exponent(a, "ocp"))
+    near = oracle.scale_exponent(a, 8.0 - 2.0 ** -20)
+    np.testing.assert_array_equal(near, oracle.scale_exponent(a, "ocp"))
+
+
+def test_qmax_at_six_never_saturates():
+    """Qmax = 6 (the largest E2M1 magnitude): every scaled element is <= 6, so no
+    element clips and the error of each element is at most half a grid step."""
+    bits, a = _all_positive_finite_bf16()
+    e = oracle.scale_exponent(a, 6.0).astype(np.int64)
+    r = np.ldexp(a, -e)
+    assert np.all(r <= 6.0)
+    deq = np.ldexp(oracle.e2m1_decode(oracle.e2m1_encode(r)), e)
+    free = e > -127
+    # grid spacing at r: 0.5 below 2, 1 in [2, 4), 2 in [4, 6]
+    step = np.where(r < 2, 0.5, np.where(r < 4, 1.0, 2.0))
+    assert np.all(np.abs(a - deq)[free] <= np.ldexp(step / 2, e)[free] * (1 + 1e-12))
+
+
+@pytest.mark.parametrize("q", [6.0, 7.5])
+def test_qmax_attention_keeps_pnq_normalization(q):
+    """PNQ's row sum is built from the quantized weights whatever the boundary:
+    V = 1 gives O = 1 exactly (to rounding)."""
+    N, d = 200, 64
+    Q, K, _ = wl.gaussian_qkv(1, 1, N, d, seed=16)
+    Q = _bits(wl.bf16_bits_to_f32(Q) * 3)
+    ones = np.full((1, 1, N, d), 0x3F80, dtype=np.uint16)
+    np.testing.assert_allclose(oracle.attention(Q, K, ones, 64, rule=q, pnq=True), 1.0, rtol=0, atol=1e-12)
+
+
+def test_qmax_rule_rejects_boundaries_outside_the_family():
+    for q in (4.0, 3.0, 8.5, 16.0):
+        with pytest.raises(ValueError):
+            oracle.scale_exponent([1.0], q)
+
+
 # ----------------------------------------------------------------------------- block quantization
 
 
