@@ -64,6 +64,17 @@ typedef enum {
 } mxattn_rule;
 
 /*
+ * Scale boundary Qmax.  The abstract names the UOS scaling boundary Qmax and
+ * chooses 7.25; the *_qmax entry points below take any boundary in (4, 8] for
+ * the same rule -- e = the smallest integer with amax <= qmax * 2^e, clamped
+ * to [-127, 127] -- so the boundary can be swept.  qmax = 8 selects the OCP
+ * rule e = floor(log2 amax) - 2, which the boundary rule approaches as qmax
+ * tends to 8 from below.  MXATTN_RULE_UOS is qmax = 7.25 and MXATTN_RULE_OCP
+ * is qmax = 8: every rule-taking call equals its *_qmax form at that value.
+ * A qmax outside (4, 8] (or NaN) returns MXATTN_ERR_INVALID.
+ */
+
+/*
  * Standalone MXFP4 quantize/pack (the abstract's "direct MXFP4 quantization";
  * the scale rule is UOS or OCP).
  *   x:      bf16 [rows, cols], cols % 32 == 0, 16-byte aligned.
@@ -74,6 +85,10 @@ typedef enum {
  */
 mxattn_status mxattn_quantize(const void* x, int64_t rows, int64_t cols, mxattn_rule rule,
                               uint8_t* codes, uint8_t* scales, mxattn_stream_t stream);
+
+/* mxattn_quantize with a scale boundary qmax in (4, 8] instead of a named rule. */
+mxattn_status mxattn_quantize_qmax(const void* x, int64_t rows, int64_t cols, float qmax, uint8_t* codes,
+                                   uint8_t* scales, mxattn_stream_t stream);
 
 /*
  * V quantize with transpose: blocks of 32 consecutive tokens of each channel
@@ -132,6 +147,20 @@ mxattn_status mxattn_prepare(const void* Q, const void* K, const void* V, int B,
                              mxattn_rule rule, void* workspace, size_t workspace_bytes, mxattn_stream_t stream);
 mxattn_status mxattn_attend(int B, int H, int N, int d, int kv_tile, int pnq, mxattn_rule rule, float softmax_scale,
                             float* O, void* workspace, size_t workspace_bytes, mxattn_stream_t stream);
+
+/*
+ * mxattn_forward / mxattn_prepare / mxattn_attend with a scale boundary qmax in
+ * (4, 8] for Q, K, V and P instead of a named rule.  Same arguments, layouts,
+ * constraints and errors otherwise; mxattn_attend_qmax must run on a workspace
+ * that mxattn_prepare_qmax filled with the same qmax.
+ */
+mxattn_status mxattn_forward_qmax(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                  int kv_tile, int pnq, float qmax, float softmax_scale, float* O, void* workspace,
+                                  size_t workspace_bytes, mxattn_stream_t stream);
+mxattn_status mxattn_prepare_qmax(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                  float qmax, void* workspace, size_t workspace_bytes, mxattn_stream_t stream);
+mxattn_status mxattn_attend_qmax(int B, int H, int N, int d, int kv_tile, int pnq, float qmax, float softmax_scale,
+                                 float* O, void* workspace, size_t workspace_bytes, mxattn_stream_t stream);
 
 /*
  * The attention step alone, on operands already quantized by the caller in

@@ -45,10 +45,35 @@ bool make_layout(int B, int H, int N, int d, Layout* L) {
     return true;
 }
 
-mxattn_status check_attention_args(int B, int H, int N, int d, int kv_tile, int pnq, mxattn_rule rule, const float* O,
-                                   const void* ws, size_t ws_bytes, Layout* L) {
+// Mantissa thresholds of the block-exponent rule for a scale boundary Qmax in
+// (4, 8]: the smallest e with amax <= Qmax * 2^e is floor(log2 amax) - 2 plus
+// one when amax's significand exceeds Qmax / 4.  Qmax = 8 is the OCP rule
+// e = floor(log2 amax) - 2 (the significand never exceeds 2).
+struct Thresholds {
+    uint32_t bf16;  // 7-bit mantissa field
+    uint32_t f32;   // 23-bit mantissa field
+};
+
+bool qmax_thresholds(float qmax, Thresholds* t) {
+    if (!(qmax > 4.f && qmax <= 8.f)) return false;  // also rejects NaN
+    const double r = static_cast<double>(qmax) / 4.0 - 1.0;  // in (0, 1]
+    t->bf16 = qmax == 8.f ? 0x7Fu : static_cast<uint32_t>(std::floor(r * 128.0));
+    t->f32 = qmax == 8.f ? 0x7FFFFFu : static_cast<uint32_t>(std::floor(r * 8388608.0));
+    return true;
+}
+
+// The boundary a named rule stands for: OCP = 8, UOS = 7.25 (the abstract's Qmax).
+bool rule_qmax(mxattn_rule rule, float* qmax) {
+    if (rule == MXATTN_RULE_OCP) *qmax = 8.f;
+    else if (rule == MXATTN_RULE_UOS) *qmax = 7.25f;
+    else return false;
+    return true;
+}
+
+mxattn_status check_attention_args(int B, int H, int N, int d, int kv_tile, int pnq, const float* O, const void* ws,
+                                   size_t ws_bytes, Layout* L) {
     if (B < 1 || H < 1 || N < 1 || O == nullptr || ws == nullptr) return MXATTN_ERR_INVALID;
-    if ((pnq != 0 && pnq != 1) || (rule != MXATTN_RULE_OCP && rule != MXATTN_RULE_UOS)) return MXATTN_ERR_INVALID;
+    if (pnq != 0 && pnq != 1) return MXATTN_ERR_INVALID;
     if (d != 64 && d != 128) return MXATTN_ERR_UNSUPPORTED;
     if (kv_tile != 64 && kv_tile != 128) return MXATTN_ERR_UNSUPPORTED;
     if (N > kMaxN || static_cast<int64_t>(B) * H > (int64_t(1) << 31) / ((N + 127) / 128))
@@ -73,10 +98,10 @@ MXATTN_API const char* mxattn_status_string(mxattn_status status) {
     return "unknown status";
 }
 
-MXATTN_API mxattn_status mxattn_quantize(const void* x, int64_t rows, int64_t cols, mxattn_rule rule, uint8_t* codes,
-                                         uint8_t* scales, mxattn_stream_t stream) {
-    if (rows < 0 || cols <= 0 || cols % 32 != 0) return MXATTN_ERR_INVALID;
-    if (rule != MXATTN_RULE_OCP && rule != MXATTN_RULE_UOS) return MXATTN_ERR_INVALID;
+MXATTN_API mxattn_status mxattn_quantize_qmax(const void* x, int64_t rows, int64_t cols, float qmax, uint8_t* codes,
+                                              uint8_t* scales, mxattn_stream_t stream) {
+    Thresholds th;
+    if (rows < 0 || cols <= 0 || cols % 32 != 0 || !qmax_thresholds(qmax, &th)) return MXATTN_ERR_INVALID;
     if (rows == 0) return MXATTN_OK;
     if (x == nullptr || codes == nullptr || scales == nullptr) return MXATTN_ERR_INVALID;
     if (!aligned(x, 16) || !aligned(codes, 4)) return MXATTN_ERR_INVALID;
@@ -84,21 +109,30 @@ MXATTN_API mxattn_status mxattn_quantize(const void* x, int64_t rows, int64_t co
     const void* xs[1] = {x};
     uint8_t* cs[1] = {codes};
     uint8_t* ss[1] = {scales};
-    cudaError_t e = mxattn::launch_quantize_rows(xs, cs, ss, 1, rows, static_cast<int>(cols), rule == MXATTN_RULE_UOS,
-                                                 0, 1, 1, 1, nullptr, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = mxattn::launch_quantize_rows(xs, cs, ss, 1, rows, static_cast<int>(cols), th.bf16, 0, 1, 1, 1,
+                                                 nullptr, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
+}
+
+MXATTN_API mxattn_status mxattn_quantize(const void* x, int64_t rows, int64_t cols, mxattn_rule rule, uint8_t* codes,
+                                         uint8_t* scales, mxattn_stream_t stream) {
+    float q;
+    if (!rule_qmax(rule, &q)) return MXATTN_ERR_INVALID;
+    return mxattn_quantize_qmax(x, rows, cols, q, codes, scales, stream);
 }
 
 MXATTN_API mxattn_status mxattn_quantize_vt(const void* v, int64_t BH, int64_t N, int64_t d, mxattn_rule rule,
                                             uint8_t* codes_t, uint8_t* scales_t, mxattn_stream_t stream) {
     if (v == nullptr || codes_t == nullptr || scales_t == nullptr || BH < 1 || N < 1) return MXATTN_ERR_INVALID;
-    if (rule != MXATTN_RULE_OCP && rule != MXATTN_RULE_UOS) return MXATTN_ERR_INVALID;
+    float q;
+    Thresholds th;
+    if (!rule_qmax(rule, &q) || !qmax_thresholds(q, &th)) return MXATTN_ERR_INVALID;
     if (d != 64 && d != 128) return MXATTN_ERR_UNSUPPORTED;
     if (N > kMaxN || BH > 65535) return MXATTN_ERR_UNSUPPORTED;
     if (!aligned(v, 16) || !aligned(codes_t, 16)) return MXATTN_ERR_INVALID;
     const int G = static_cast<int>((N + 127) / 128);
-    cudaError_t e = mxattn::launch_quantize_vt(v, BH, static_cast<int>(N), static_cast<int>(d), rule == MXATTN_RULE_UOS,
-                                               0, G, codes_t, scales_t, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = mxattn::launch_quantize_vt(v, BH, static_cast<int>(N), static_cast<int>(d), th.bf16, 0,
+                                               G, codes_t, scales_t, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
 }
 
@@ -107,12 +141,14 @@ MXATTN_API size_t mxattn_workspace_size(int B, int H, int N, int d) {
     return make_layout(B, H, N, d, &L) ? L.total : 0;
 }
 
-MXATTN_API mxattn_status mxattn_prepare(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
-                                        mxattn_rule rule, void* workspace, size_t workspace_bytes,
-                                        mxattn_stream_t stream) {
+MXATTN_API mxattn_status mxattn_prepare_qmax(const void* Q, const void* K, const void* V, int B, int H, int N,
+                                             int d, float qmax, void* workspace, size_t workspace_bytes,
+                                             mxattn_stream_t stream) {
     Layout L;
     float dummy_out[4];
-    mxattn_status st = check_attention_args(B, H, N, d, 128, 1, rule, dummy_out, workspace, workspace_bytes, &L);
+    Thresholds th;
+    if (!qmax_thresholds(qmax, &th)) return MXATTN_ERR_INVALID;
+    mxattn_status st = check_attention_args(B, H, N, d, 128, 1, dummy_out, workspace, workspace_bytes, &L);
     if (st != MXATTN_OK) return st;
     if (Q == nullptr || K == nullptr || V == nullptr) return MXATTN_ERR_INVALID;
     if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16)) return MXATTN_ERR_INVALID;
@@ -122,21 +158,30 @@ MXATTN_API mxattn_status mxattn_prepare(const void* Q, const void* K, const void
     uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
     const int64_t BH = static_cast<int64_t>(B) * H;
     const int G = (N + 127) / 128;
-    const int uos = rule == MXATTN_RULE_UOS;
     const void* xs[2] = {Q, K};
     uint8_t* cs[2] = {ws + L.q_codes, ws + L.k_codes};
     uint8_t* ss[2] = {ws + L.q_sf, ws + L.k_sf};
-    cudaError_t e = mxattn::launch_quantize_rows(xs, cs, ss, 2, BH * N, d, uos, 1, N, G, BH, status, s);
+    cudaError_t e = mxattn::launch_quantize_rows(xs, cs, ss, 2, BH * N, d, th.bf16, 1, N, G, BH, status, s);
     if (e != cudaSuccess) return MXATTN_ERR_CUDA;
-    e = mxattn::launch_quantize_vt(V, BH, N, d, uos, 1, G, ws + L.vt_codes, ws + L.v_sf, s);
+    e = mxattn::launch_quantize_vt(V, BH, N, d, th.bf16, 1, G, ws + L.vt_codes, ws + L.v_sf, s);
     return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
 }
 
-MXATTN_API mxattn_status mxattn_attend(int B, int H, int N, int d, int kv_tile, int pnq, mxattn_rule rule,
-                                       float softmax_scale, float* O, void* workspace, size_t workspace_bytes,
-                                       mxattn_stream_t stream) {
+MXATTN_API mxattn_status mxattn_prepare(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                        mxattn_rule rule, void* workspace, size_t workspace_bytes,
+                                        mxattn_stream_t stream) {
+    float q;
+    if (!rule_qmax(rule, &q)) return MXATTN_ERR_INVALID;
+    return mxattn_prepare_qmax(Q, K, V, B, H, N, d, q, workspace, workspace_bytes, stream);
+}
+
+MXATTN_API mxattn_status mxattn_attend_qmax(int B, int H, int N, int d, int kv_tile, int pnq, float qmax,
+                                            float softmax_scale, float* O, void* workspace, size_t workspace_bytes,
+                                            mxattn_stream_t stream) {
     Layout L;
-    mxattn_status st = check_attention_args(B, H, N, d, kv_tile, pnq, rule, O, workspace, workspace_bytes, &L);
+    Thresholds th;
+    if (!qmax_thresholds(qmax, &th)) return MXATTN_ERR_INVALID;
+    mxattn_status st = check_attention_args(B, H, N, d, kv_tile, pnq, O, workspace, workspace_bytes, &L);
     if (st != MXATTN_OK) return st;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     mxattn::AttnArgs a{};
@@ -153,21 +198,40 @@ MXATTN_API mxattn_status mxattn_attend(int B, int H, int N, int d, int kv_tile, 
     a.d = d;
     a.kv_tile = kv_tile;
     a.pnq = pnq;
-    a.uos = rule == MXATTN_RULE_UOS;
+    a.p_thresh = th.f32;
     a.softmax_scale = resolve_scale(softmax_scale, d);
     cudaError_t e = mxattn::launch_attention(a, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
 }
 
+MXATTN_API mxattn_status mxattn_attend(int B, int H, int N, int d, int kv_tile, int pnq, mxattn_rule rule,
+                                       float softmax_scale, float* O, void* workspace, size_t workspace_bytes,
+                                       mxattn_stream_t stream) {
+    float q;
+    if (!rule_qmax(rule, &q)) return MXATTN_ERR_INVALID;
+    return mxattn_attend_qmax(B, H, N, d, kv_tile, pnq, q, softmax_scale, O, workspace, workspace_bytes, stream);
+}
+
+MXATTN_API mxattn_status mxattn_forward_qmax(const void* Q, const void* K, const void* V, int B, int H, int N,
+                                             int d, int kv_tile, int pnq, float qmax, float softmax_scale, float* O,
+                                             void* workspace, size_t workspace_bytes, mxattn_stream_t stream) {
+    Layout L;
+    Thresholds th;
+    if (!qmax_thresholds(qmax, &th)) return MXATTN_ERR_INVALID;
+    mxattn_status st = check_attention_args(B, H, N, d, kv_tile, pnq, O, workspace, workspace_bytes, &L);
+    if (st != MXATTN_OK) return st;
+    st = mxattn_prepare_qmax(Q, K, V, B, H, N, d, qmax, workspace, workspace_bytes, stream);
+    if (st != MXATTN_OK) return st;
+    return mxattn_attend_qmax(B, H, N, d, kv_tile, pnq, qmax, softmax_scale, O, workspace, workspace_bytes, stream);
+}
+
 MXATTN_API mxattn_status mxattn_forward(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
                                         int kv_tile, int pnq, mxattn_rule rule, float softmax_scale, float* O,
                                         void* workspace, size_t workspace_bytes, mxattn_stream_t stream) {
-    Layout L;
-    mxattn_status st = check_attention_args(B, H, N, d, kv_tile, pnq, rule, O, workspace, workspace_bytes, &L);
-    if (st != MXATTN_OK) return st;
-    st = mxattn_prepare(Q, K, V, B, H, N, d, rule, workspace, workspace_bytes, stream);
-    if (st != MXATTN_OK) return st;
-    return mxattn_attend(B, H, N, d, kv_tile, pnq, rule, softmax_scale, O, workspace, workspace_bytes, stream);
+    float q;
+    if (!rule_qmax(rule, &q)) return MXATTN_ERR_INVALID;
+    return mxattn_forward_qmax(Q, K, V, B, H, N, d, kv_tile, pnq, q, softmax_scale, O, workspace, workspace_bytes,
+                               stream);
 }
 
 MXATTN_API mxattn_status mxattn_forward_quantized(const uint8_t* q_codes, const uint8_t* q_scales,
@@ -177,7 +241,10 @@ MXATTN_API mxattn_status mxattn_forward_quantized(const uint8_t* q_codes, const 
                                                   float softmax_scale, float* O, void* workspace,
                                                   size_t workspace_bytes, mxattn_stream_t stream) {
     Layout L;
-    mxattn_status st = check_attention_args(B, H, N, d, kv_tile, pnq, rule, O, workspace, workspace_bytes, &L);
+    float q;
+    Thresholds th;
+    if (!rule_qmax(rule, &q) || !qmax_thresholds(q, &th)) return MXATTN_ERR_INVALID;
+    mxattn_status st = check_attention_args(B, H, N, d, kv_tile, pnq, O, workspace, workspace_bytes, &L);
     if (st != MXATTN_OK) return st;
     if (!q_codes || !q_scales || !k_codes || !k_scales || !vt_codes || !vt_scales) return MXATTN_ERR_INVALID;
     if (!aligned(q_codes, 16) || !aligned(k_codes, 16) || !aligned(vt_codes, 16)) return MXATTN_ERR_INVALID;
@@ -203,7 +270,7 @@ MXATTN_API mxattn_status mxattn_forward_quantized(const uint8_t* q_codes, const 
     a.d = d;
     a.kv_tile = kv_tile;
     a.pnq = pnq;
-    a.uos = rule == MXATTN_RULE_UOS;
+    a.p_thresh = th.f32;
     a.softmax_scale = resolve_scale(softmax_scale, d);
     e = mxattn::launch_attention(a, s);
     return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;

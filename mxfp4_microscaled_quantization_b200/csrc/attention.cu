@@ -133,7 +133,7 @@ struct KParams {
     int nq2;     // CTAs (pairs of query tiles) per head
     int nkv;     // key tiles per head
     int groups;  // 128-row scale groups per head
-    int uos;
+    uint32_t p_thresh;  // block exponent of P: mantissa threshold of the scale boundary
     float kq;    // softmax_scale * log2(e)
 };
 
@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t t_o = tbase + lane_base + C::kColO + t * C::kOCols;
         const float kq = p.kq;
-        const int uos = p.uos;
+        const uint32_t p_thresh = p.p_thresh;
         const int valid_last = p.N - (nkv - 1) * T;
         uint8_t* sPt = sP + t * C::kPBytes;
         uint8_t* sPsft = sPsf + t * 512;
@@ -436,7 +436,7 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
 #pragma unroll
             for (int k = 0; k < T / 32; ++k) {
                 const float pmax = ex2_approx((bm[k] - m_new) * kq);
-                const int e = block_exponent_f32(__float_as_uint(pmax), uos);
+                const int e = block_exponent_f32(__float_as_uint(pmax), p_thresh);
                 const float nbias = -fmaf(m_new, kq, static_cast<float>(e));
                 float bsum = 0.f;
 #pragma unroll
@@ -587,7 +587,7 @@ cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
     kp.nq2 = (a.N + C::kRows - 1) / C::kRows;
     kp.nkv = (a.N + T - 1) / T;
     kp.groups = (a.N + 127) / 128;
-    kp.uos = a.uos;
+    kp.p_thresh = a.p_thresh;
     kp.kq = static_cast<float>(static_cast<double>(a.softmax_scale) * 1.4426950408889634);
     dim3 grid(static_cast<unsigned>(a.BH * kp.nq2));
     mxattn_fwd_kernel<D, T, PNQ><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, kp);

@@ -13,12 +13,12 @@ namespace mxattn {
 // the 128-row regrouped order (padding rows zeroed).  Clears *status when
 // status != nullptr.
 cudaError_t launch_quantize_rows(const void* const* x, uint8_t* const* codes, uint8_t* const* scales, int ntensors,
-                                 int64_t rows, int cols, int uos, int regroup, int N, int groups, int64_t BH,
+                                 int64_t rows, int cols, uint32_t sf_thresh, int regroup, int N, int groups, int64_t BH,
                                  uint32_t* status, cudaStream_t stream);
 
 // V [BH, N, d] -> V^T codes [BH, d, Npad/2] and scales (row-major
 // [BH, d, Npad/32] when regroup = 0, regrouped per 128 tokens when 1).
-cudaError_t launch_quantize_vt(const void* v, int64_t BH, int N, int d, int uos, int regroup, int groups,
+cudaError_t launch_quantize_vt(const void* v, int64_t BH, int N, int d, uint32_t sf_thresh, int regroup, int groups,
                                uint8_t* codes_t, uint8_t* scales_t, cudaStream_t stream);
 
 // Row-major Q/K/V^T scales -> regrouped scales; clears *status.
@@ -40,7 +40,7 @@ struct AttnArgs {
     int d;
     int kv_tile;
     int pnq;
-    int uos;
+    uint32_t p_thresh;  // block-exponent mantissa threshold for P (fp32 bits)
     float softmax_scale;
 };
 

@@ -401,22 +401,25 @@ __device__ __forceinline__ uint32_t pack_e2m1x8(const float (&x)[8]) {
     return out;
 }
 
-// Block exponent from the fp32 bit pattern of the block maximum (>= 0).
-//   OCP: floor(log2 amax) - 2.   UOS: smallest e with amax <= 7.25 * 2^e,
-//   i.e. the OCP value plus one when the significand exceeds 1.8125
-//   (mantissa field > 0x680000).  Zero and subnormal maxima give -127.
-__device__ __forceinline__ int block_exponent_f32(uint32_t amax_bits, int uos) {
+// Block exponent from the fp32 bit pattern of the block maximum (>= 0) under
+// a scale boundary Qmax in (4, 8]: the smallest e with amax <= Qmax * 2^e is
+// floor(log2 amax) - 2, plus one when the significand exceeds Qmax / 4, i.e.
+// when the mantissa field exceeds `mant_thresh` = floor((Qmax/4 - 1) * 2^23).
+//   UOS (Qmax = 7.25): 0x680000.   OCP (floor(log2 amax) - 2): 0x7FFFFF, never
+//   exceeded.  Zero and subnormal maxima give -127.
+__device__ __forceinline__ int block_exponent_f32(uint32_t amax_bits, uint32_t mant_thresh) {
     const int E = static_cast<int>((amax_bits >> 23) & 0xFFu);
     if (E == 0) return -127;
-    int e = E - 129 + ((uos && (amax_bits & 0x7FFFFFu) > 0x680000u) ? 1 : 0);
+    int e = E - 129 + (((amax_bits & 0x7FFFFFu) > mant_thresh) ? 1 : 0);
     return e < -127 ? -127 : (e > 127 ? 127 : e);
 }
 
-// Same rule on a bfloat16 bit pattern (mantissa field > 0x68 for UOS).
-__device__ __forceinline__ int block_exponent_bf16(uint32_t amax_bits, int uos) {
+// Same rule on a bfloat16 bit pattern: mantissa field > floor((Qmax/4 - 1) * 2^7)
+// (UOS: 0x68; OCP: 0x7F, never exceeded).
+__device__ __forceinline__ int block_exponent_bf16(uint32_t amax_bits, uint32_t mant_thresh) {
     const int E = static_cast<int>((amax_bits >> 7) & 0xFFu);
     if (E == 0) return -127;
-    int e = E - 129 + ((uos && (amax_bits & 0x7Fu) > 0x68u) ? 1 : 0);
+    int e = E - 129 + (((amax_bits & 0x7Fu) > mant_thresh) ? 1 : 0);
     return e < -127 ? -127 : (e > 127 ? 127 : e);
 }
 

@@ -41,7 +41,7 @@ constexpr int kCtasPerSm = MXATTN_QUANT_CTAS_PER_SM;     // grid of the grid-str
 
 // One 32-element block spread over a quad of lanes (8 elements each).
 // Returns the packed codes of this lane's 8 elements; `e_out` gets the block exponent.
-__device__ __forceinline__ uint32_t quantize_quad(uint4 raw, int uos, int& e_out) {
+__device__ __forceinline__ uint32_t quantize_quad(uint4 raw, uint32_t sf_thresh, int& e_out) {
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
     uint32_t amax = 0;
 #pragma unroll
@@ -51,7 +51,7 @@ __device__ __forceinline__ uint32_t quantize_quad(uint4 raw, int uos, int& e_out
     }
     amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    const int e = block_exponent_bf16(amax, uos);
+    const int e = block_exponent_bf16(amax, sf_thresh);
     const float sc = exp2_neg_int(e);
     float f[8];
 #pragma unroll
@@ -71,7 +71,7 @@ struct RowsArgs {
 
 // Row quantization with row-major scales [rows, cols/32] (the standalone op):
 // grid-stride over 16-byte chunks, kUnroll loads in flight per lane.
-__global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(RowsArgs a, int64_t n_chunks, int cols, int uos,
+__global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(RowsArgs a, int64_t n_chunks, int cols, uint32_t sf_thresh,
                                                                       uint32_t* status) {
     const uint16_t* __restrict__ x = a.x[0];
     uint32_t* __restrict__ codes = reinterpret_cast<uint32_t*>(a.codes[0]);
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(RowsArgs a
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t i = base + u * 32 + lane;
             int e;
-            const uint32_t packed = quantize_quad(raw[u], uos, e);
+            const uint32_t packed = quantize_quad(raw[u], sf_thresh, e);
             if (i < n_chunks) {
                 codes[i] = packed;
                 if ((lane & 3) == 0) scales[i >> 2] = static_cast<uint8_t>(e + 127);
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(RowsArgs a
 // past N are zeros; the group's 512 scale bytes are assembled in shared memory
 // in the regrouped order and written out contiguously.
 template <int D>
-__global__ void __launch_bounds__(kQuantThreads) quantize_rows_grouped_kernel(RowsArgs a, int N, int groups, int uos,
+__global__ void __launch_bounds__(kQuantThreads) quantize_rows_grouped_kernel(RowsArgs a, int N, int groups, uint32_t sf_thresh,
                                                                               uint32_t* status) {
     constexpr int kChunksPerRow = D / 8;                          // 16-byte chunks per row
     constexpr int kPerThread = 128 * kChunksPerRow / kQuantThreads;
@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_grouped_kernel(Ro
         const int c = threadIdx.x + u * kQuantThreads;
         const int m = c / kChunksPerRow;
         int e;
-        const uint32_t packed = quantize_quad(raw[u], uos, e);
+        const uint32_t packed = quantize_quad(raw[u], sf_thresh, e);
         if (m < rows_valid) codes[(row0 + m) * (D / 8) + (c % kChunksPerRow)] = packed;
         if ((threadIdx.x & 3) == 0) {
             const int k = (c % kChunksPerRow) / 4;
@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_grouped_kernel(Ro
 // 128 tokens x D channels (bf16) in shared memory; thread `ch` then quantizes
 // the four 32-token blocks of its channel and writes 64 contiguous code bytes.
 template <int D>
-__global__ void __launch_bounds__(D) quantize_vt_kernel(const uint16_t* __restrict__ v, int N, int npad, int uos,
+__global__ void __launch_bounds__(D) quantize_vt_kernel(const uint16_t* __restrict__ v, int N, int npad, uint32_t sf_thresh,
                                                         int regroup, int groups, uint8_t* __restrict__ codes_t,
                                                         uint8_t* __restrict__ scales_t) {
     __shared__ __align__(16) uint16_t tile[128 * D];
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(D) quantize_vt_kernel(const uint16_t* __restri
             raw[i] = tile[(32 * k + i) * D + ch];
             amax = max(amax, raw[i] & 0x7FFFu);
         }
-        const int e = block_exponent_bf16(amax, uos);
+        const int e = block_exponent_bf16(amax, sf_thresh);
         const float sc = exp2_neg_int(e);
         uint32_t words[4];
 #pragma unroll
@@ -259,7 +259,7 @@ int grid_for(int64_t work_items, int per_block) {
 }  // namespace
 
 cudaError_t launch_quantize_rows(const void* const* x, uint8_t* const* codes, uint8_t* const* scales, int ntensors,
-                                 int64_t rows, int cols, int uos, int regroup, int N, int groups, int64_t BH,
+                                 int64_t rows, int cols, uint32_t sf_thresh, int regroup, int N, int groups, int64_t BH,
                                  uint32_t* status, cudaStream_t stream) {
     RowsArgs a{};
     for (int t = 0; t < ntensors; ++t) {
@@ -270,26 +270,26 @@ cudaError_t launch_quantize_rows(const void* const* x, uint8_t* const* codes, ui
     if (regroup) {
         dim3 grid(groups, static_cast<unsigned>(BH), ntensors);
         if (cols == 128)
-            quantize_rows_grouped_kernel<128><<<grid, kQuantThreads, 0, stream>>>(a, N, groups, uos, status);
+            quantize_rows_grouped_kernel<128><<<grid, kQuantThreads, 0, stream>>>(a, N, groups, sf_thresh, status);
         else
-            quantize_rows_grouped_kernel<64><<<grid, kQuantThreads, 0, stream>>>(a, N, groups, uos, status);
+            quantize_rows_grouped_kernel<64><<<grid, kQuantThreads, 0, stream>>>(a, N, groups, sf_thresh, status);
         return cudaGetLastError();
     }
     const int64_t n_chunks = rows * cols / 8;
     dim3 grid(grid_for(n_chunks / kUnroll, kQuantThreads), ntensors);
-    quantize_rows_kernel<<<grid, kQuantThreads, 0, stream>>>(a, n_chunks, cols, uos, status);
+    quantize_rows_kernel<<<grid, kQuantThreads, 0, stream>>>(a, n_chunks, cols, sf_thresh, status);
     return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_vt(const void* v, int64_t BH, int N, int d, int uos, int regroup, int groups,
+cudaError_t launch_quantize_vt(const void* v, int64_t BH, int N, int d, uint32_t sf_thresh, int regroup, int groups,
                                uint8_t* codes_t, uint8_t* scales_t, cudaStream_t stream) {
     const int npad = (N + 31) / 32 * 32;
     dim3 grid(groups, static_cast<unsigned>(BH));
     if (d == 128)
-        quantize_vt_kernel<128><<<grid, 128, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, uos, regroup,
+        quantize_vt_kernel<128><<<grid, 128, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, sf_thresh, regroup,
                                                            groups, codes_t, scales_t);
     else
-        quantize_vt_kernel<64><<<grid, 64, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, uos, regroup, groups,
+        quantize_vt_kernel<64><<<grid, 64, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, sf_thresh, regroup, groups,
                                                          codes_t, scales_t);
     return cudaGetLastError();
 }

@@ -58,6 +58,15 @@ def lib() -> ctypes.CDLL:
         L.mxattn_forward_quantized.restype = i32
         L.mxattn_forward_noalloc.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, ctypes.c_float, P, P]
         L.mxattn_forward_noalloc.restype = i32
+        f32 = ctypes.c_float
+        L.mxattn_quantize_qmax.argtypes = [P, i64, i64, f32, P, P, P]
+        L.mxattn_quantize_qmax.restype = i32
+        L.mxattn_forward_qmax.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f32, f32, P, P, u64, P]
+        L.mxattn_forward_qmax.restype = i32
+        L.mxattn_prepare_qmax.argtypes = [P, P, P, i32, i32, i32, i32, f32, P, u64, P]
+        L.mxattn_prepare_qmax.restype = i32
+        L.mxattn_attend_qmax.argtypes = [i32, i32, i32, i32, i32, i32, f32, f32, P, P, u64, P]
+        L.mxattn_attend_qmax.restype = i32
         L.mxattn_workspace_status.argtypes = [P, P]
         L.mxattn_workspace_status.restype = i32
         L.mxattn_wait_selftest.argtypes = [i32, ctypes.c_uint, P, P]
@@ -83,7 +92,15 @@ def _check(status: int, where: str):
 
 
 def _rule(rule) -> int:
-    return RULES[rule] if isinstance(rule, str) else int(rule)
+    if not isinstance(rule, str):
+        raise ValueError(f"this call takes a named rule ('ocp' or 'uos'), got {rule!r}")
+    return RULES[rule]
+
+
+def _qmax(rule):
+    """None for a named rule ('ocp', 'uos'); else the scale boundary Qmax in (4, 8]
+    (checked by the library) for the *_qmax entry points."""
+    return None if isinstance(rule, str) else float(rule)
 
 
 def _stream(stream):
@@ -112,8 +129,13 @@ def mxattn_quantize(x: torch.Tensor, rule="uos", codes=None, scales=None, stream
         codes = torch.empty(x.shape[:-1] + (cols // 2,), dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty(x.shape[:-1] + (cols // 32,), dtype=torch.uint8, device=x.device)
-    _check(lib().mxattn_quantize(_cuda(x, "x", torch.bfloat16), rows, cols, _rule(rule), _cuda(codes, "codes"),
-                                 _cuda(scales, "scales"), _stream(stream)), "mxattn_quantize")
+    q = _qmax(rule)
+    if q is None:
+        _check(lib().mxattn_quantize(_cuda(x, "x", torch.bfloat16), rows, cols, _rule(rule), _cuda(codes, "codes"),
+                                     _cuda(scales, "scales"), _stream(stream)), "mxattn_quantize")
+    else:
+        _check(lib().mxattn_quantize_qmax(_cuda(x, "x", torch.bfloat16), rows, cols, q, _cuda(codes, "codes"),
+                                          _cuda(scales, "scales"), _stream(stream)), "mxattn_quantize_qmax")
     return codes, scales
 
 
@@ -159,7 +181,8 @@ def new_workspace(B, H, N, d, device="cuda") -> torch.Tensor:
 
 def mxattn_forward(q, k, v, kv_tile=128, pnq=True, rule="uos", softmax_scale=0.0, out=None, workspace=None,
                    stream=None):
-    """Fused MXFP4 attention: q, k, v bf16 [B, H, N, d] -> O fp32 [B, H, N, d]."""
+    """Fused MXFP4 attention: q, k, v bf16 [B, H, N, d] -> O fp32 [B, H, N, d].
+    `rule`: "uos", "ocp", or a scale boundary Qmax in (4, 8] (mxattn_forward_qmax)."""
     B, H, N, d = q.shape
     if k.shape != q.shape or v.shape != q.shape:
         raise ValueError("q, k, v must have the same shape [B, H, N, d]")
@@ -167,10 +190,13 @@ def mxattn_forward(q, k, v, kv_tile=128, pnq=True, rule="uos", softmax_scale=0.0
         out = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
     if workspace is None:
         workspace = new_workspace(B, H, N, d, q.device)
-    _check(lib().mxattn_forward(_cuda(q, "q", torch.bfloat16), _cuda(k, "k", torch.bfloat16),
-                                _cuda(v, "v", torch.bfloat16), B, H, N, d, kv_tile, 1 if pnq else 0, _rule(rule),
-                                float(softmax_scale), _cuda(out, "out", torch.float32), _cuda(workspace, "workspace"),
-                                workspace.numel(), _stream(stream)), "mxattn_forward")
+    qm = _qmax(rule)
+    fn, name = (lib().mxattn_forward, "mxattn_forward") if qm is None else (lib().mxattn_forward_qmax,
+                                                                             "mxattn_forward_qmax")
+    _check(fn(_cuda(q, "q", torch.bfloat16), _cuda(k, "k", torch.bfloat16), _cuda(v, "v", torch.bfloat16), B, H, N, d,
+              kv_tile, 1 if pnq else 0, _rule(rule) if qm is None else qm, float(softmax_scale),
+              _cuda(out, "out", torch.float32), _cuda(workspace, "workspace"), workspace.numel(), _stream(stream)),
+           name)
     return out
 
 
@@ -181,9 +207,12 @@ def mxattn_prepare(q, k, v, rule="uos", workspace=None, stream=None):
         raise ValueError("q, k, v must have the same shape [B, H, N, d]")
     if workspace is None:
         workspace = new_workspace(B, H, N, d, q.device)
-    _check(lib().mxattn_prepare(_cuda(q, "q", torch.bfloat16), _cuda(k, "k", torch.bfloat16),
-                                _cuda(v, "v", torch.bfloat16), B, H, N, d, _rule(rule), _cuda(workspace, "workspace"),
-                                workspace.numel(), _stream(stream)), "mxattn_prepare")
+    qm = _qmax(rule)
+    fn, name = (lib().mxattn_prepare, "mxattn_prepare") if qm is None else (lib().mxattn_prepare_qmax,
+                                                                             "mxattn_prepare_qmax")
+    _check(fn(_cuda(q, "q", torch.bfloat16), _cuda(k, "k", torch.bfloat16), _cuda(v, "v", torch.bfloat16), B, H, N, d,
+              _rule(rule) if qm is None else qm, _cuda(workspace, "workspace"), workspace.numel(), _stream(stream)),
+           name)
     return workspace
 
 
@@ -191,9 +220,12 @@ def mxattn_attend(workspace, B, H, N, d, kv_tile=128, pnq=True, rule="uos", soft
     """Attention on a workspace filled by mxattn_prepare (the second half of mxattn_forward)."""
     if out is None:
         out = torch.empty((B, H, N, d), dtype=torch.float32, device=workspace.device)
-    _check(lib().mxattn_attend(B, H, N, d, kv_tile, 1 if pnq else 0, _rule(rule), float(softmax_scale),
-                               _cuda(out, "out", torch.float32), _cuda(workspace, "workspace"), workspace.numel(),
-                               _stream(stream)), "mxattn_attend")
+    qm = _qmax(rule)
+    fn, name = (lib().mxattn_attend, "mxattn_attend") if qm is None else (lib().mxattn_attend_qmax,
+                                                                           "mxattn_attend_qmax")
+    _check(fn(B, H, N, d, kv_tile, 1 if pnq else 0, _rule(rule) if qm is None else qm, float(softmax_scale),
+              _cuda(out, "out", torch.float32), _cuda(workspace, "workspace"), workspace.numel(), _stream(stream)),
+           name)
     return out
 
 

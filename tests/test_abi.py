@@ -85,3 +85,17 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(mx, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         mx.lib()
+
+
+def test_qmax_entry_points_reject_boundaries_outside_the_family(L):
+    """A scale boundary outside (4, 8] (or NaN) is an argument error, caught before any launch."""
+    fake = _p(1 << 20)
+    f = ctypes.c_float
+    ws_ok = mx.mxattn_workspace_size(1, 1, 256, 64)
+    for q in (4.0, 3.0, 8.5, float("nan"), -7.25):
+        assert L.mxattn_quantize_qmax(fake, 4, 64, f(q), fake, fake, None) == 1
+        assert L.mxattn_forward_qmax(fake, fake, fake, 1, 1, 256, 64, 64, 1, f(q), f(0.0), fake, fake, ws_ok,
+                                     None) == 1
+        assert L.mxattn_prepare_qmax(fake, fake, fake, 1, 1, 256, 64, f(q), fake, ws_ok, None) == 1
+        assert L.mxattn_attend_qmax(1, 1, 256, 64, 64, 1, f(q), f(0.0), fake, fake, ws_ok, None) == 1
+    assert L.mxattn_quantize_qmax(None, 0, 64, f(6.0), None, None, None) == 0  # empty, valid boundary
