@@ -51,14 +51,12 @@ bool make_layout(int B, int H, int N, int d, Layout* L) {
 // e = floor(log2 amax) - 2 (the significand never exceeds 2).
 struct Thresholds {
     uint32_t bf16;  // 7-bit mantissa field
-    uint32_t f32;   // 23-bit mantissa field
 };
 
 bool qmax_thresholds(float qmax, Thresholds* t) {
     if (!(qmax > 4.f && qmax <= 8.f)) return false;  // also rejects NaN
     const double r = static_cast<double>(qmax) / 4.0 - 1.0;  // in (0, 1]
     t->bf16 = qmax == 8.f ? 0x7Fu : static_cast<uint32_t>(std::floor(r * 128.0));
-    t->f32 = qmax == 8.f ? 0x7FFFFFu : static_cast<uint32_t>(std::floor(r * 8388608.0));
     return true;
 }
 
@@ -198,7 +196,7 @@ MXATTN_API mxattn_status mxattn_attend_qmax(int B, int H, int N, int d, int kv_t
     a.d = d;
     a.kv_tile = kv_tile;
     a.pnq = pnq;
-    a.p_thresh = th.f32;
+    a.qmax = qmax;
     a.softmax_scale = resolve_scale(softmax_scale, d);
     cudaError_t e = mxattn::launch_attention(a, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
@@ -270,7 +268,7 @@ MXATTN_API mxattn_status mxattn_forward_quantized(const uint8_t* q_codes, const 
     a.d = d;
     a.kv_tile = kv_tile;
     a.pnq = pnq;
-    a.p_thresh = th.f32;
+    a.qmax = q;
     a.softmax_scale = resolve_scale(softmax_scale, d);
     e = mxattn::launch_attention(a, s);
     return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;

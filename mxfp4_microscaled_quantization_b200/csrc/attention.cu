@@ -50,9 +50,6 @@ namespace {
 
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
 constexpr uint32_t kTimeoutCode = 4u;           // MXATTN_ERR_TIMEOUT
-#ifndef MXATTN_FMA_EXP_PAIRS
-#define MXATTN_FMA_EXP_PAIRS 1
-#endif
 #ifndef MXATTN_ROLE_WAIT_HINT_NS
 #define MXATTN_ROLE_WAIT_HINT_NS 0
 #endif
@@ -85,7 +82,14 @@ struct Cfg {
     static constexpr int kPBytes = 128 * T / 2;
     static constexpr int kSfBytes = 512;
     static constexpr int kOCols = D + 16;
-    static constexpr int kFmaExpPairs = MXATTN_FMA_EXP_PAIRS;  // of every 4 exponential pairs, this many use the FMA pipe
+    // Of the 16 exponential pairs of a 32-column block, this many go to the FMA
+    // pipe instead of the MUFU: 7 with PNQ (the code-only stand-in for 2^w,
+    // exp2_code_x2), 6 without (the full polynomial, exp2_fma_x2); pair q is
+    // one of them when (q * n) mod 16 < n, which spreads them evenly.
+    __host__ __device__ static constexpr bool fma_pair(int q, bool pnq) {
+        const int n = pnq ? 7 : 6;
+        return (q * n) % 16 < n;
+    }
 
     static constexpr uint32_t kQKLayout = (D == 128) ? kLayoutSw64 : kLayoutSw32;
     static constexpr uint32_t kQKSbo = 8 * D / 2;
@@ -133,8 +137,15 @@ struct KParams {
     int nq2;     // CTAs (pairs of query tiles) per head
     int nkv;     // key tiles per head
     int groups;  // 128-row scale groups per head
-    uint32_t p_thresh;  // block exponent of P: mantissa threshold of the scale boundary
     float kq;    // softmax_scale * log2(e)
+    // Block exponent of P in the log domain: e = sign * floor(sign * x + off) + add
+    // with x = log2 of the block's largest exponential.  Boundary Qmax < 8:
+    // sign = -1, off = log2(Qmax), add = 0, so e = ceil(x - log2 Qmax), the
+    // smallest e with 2^x <= Qmax * 2^e.  OCP (Qmax = 8): sign = +1, off = 0,
+    // add = -2, so e = floor(x) - 2 (floor of x itself, exact at integer x).
+    float e_sign;
+    float e_off;
+    int e_add;
 };
 
 // Maximum of 32 values as a depth-4 tree of 3-input max instructions.
@@ -389,7 +400,9 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t t_o = tbase + lane_base + C::kColO + t * C::kOCols;
         const float kq = p.kq;
-        const uint32_t p_thresh = p.p_thresh;
+        const float e_sign = p.e_sign;
+        const float e_off = p.e_off;
+        const int e_add = p.e_add;
         const int valid_last = p.N - (nkv - 1) * T;
         uint8_t* sPt = sP + t * C::kPBytes;
         uint8_t* sPsft = sPsf + t * 512;
@@ -403,14 +416,14 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                 break;
             }
             tc_fence_after_sync();
+            uint32_t sr[T / 64][64];
+#pragma unroll
+            for (int c = 0; c < T / 64; ++c) tmem_ld64_sync(tbase + lane_base + C::kColS + 64 * c, sr[c]);
             float sv[T];
 #pragma unroll
-            for (int c = 0; c < T / 64; ++c) {
-                uint32_t r[64];
-                tmem_ld64_sync(tbase + lane_base + C::kColS + 64 * c, r);
+            for (int c = 0; c < T / 64; ++c)
 #pragma unroll
-                for (int i = 0; i < 64; ++i) sv[64 * c + i] = __uint_as_float(r[i]);
-            }
+                for (int i = 0; i < 64; ++i) sv[64 * c + i] = __uint_as_float(sr[c][i]);
             tc_fence_before_sync();
             mbar_arrive(bar_s_loaded + t);
             if (j == nkv - 1 && valid_last < T) {
@@ -428,15 +441,22 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
             const bool rescale = (j > 0) && (m_new > m_run);
             const float alpha = rescale ? ex2_approx((m_run - m_new) * kq) : 1.f;
 
-            // PNQ: quantize exp(S - m_new) per 32-column block.  pmax = 2^((bm - m) * kq)
-            // gives the block exponent e; each element is then 2^(s*kq - (m*kq + e)).
+            // PNQ: quantize exp(S - m_new) per 32-column block.  The block's largest
+            // exponential is 2^x with x = (bm - m_new) * kq; the scale rule is applied to
+            // it in the log domain (no exponential needed), and each element is then
+            // 2^(s*kq - (m*kq + e)), already divided by the block scale 2^e.
             uint32_t pw[T / 8];
             uint32_t sfw = 0;
             float lsum = 0.f;
 #pragma unroll
             for (int k = 0; k < T / 32; ++k) {
-                const float pmax = ex2_approx((bm[k] - m_new) * kq);
-                const int e = block_exponent_f32(__float_as_uint(pmax), p_thresh);
+                // x = (bm - m_new) * kq is exactly 0 for the block holding the row max, so
+                // the OCP boundary at integer x is decided exactly there.
+                float z = fmaf(e_sign, (bm[k] - m_new) * kq, e_off);
+                z = fminf(fmaxf(z, -250.f), 250.f);  // masked blocks give +-inf; any |z| > 127 clamps e below
+                const int fl = static_cast<int>(__float_as_uint(__fadd_rd(z, 12582912.f)) - 0x4B400000u);
+                int e = (e_sign > 0.f ? fl : -fl) + e_add;
+                e = e < -127 ? -127 : e;
                 const float nbias = -fmaf(m_new, kq, static_cast<float>(e));
                 float bsum = 0.f;
 #pragma unroll
@@ -446,10 +466,12 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                     for (int i = 0; i < 8; i += 2) {
                         float w0, w1;
                         ffma2_bcast(w0, w1, sv[32 * k + 8 * g + i], sv[32 * k + 8 * g + i + 1], kq, nbias);
-                        if (i / 2 < 4 - C::kFmaExpPairs) {  // MUFU
+                        if (!C::fma_pair(4 * g + i / 2, PNQ)) {  // MUFU
                             f[i] = ex2_approx(w0);
                             f[i + 1] = ex2_approx(w1);
-                        } else {                            // FMA pipe
+                        } else if constexpr (PNQ) {  // FMA pipe: only the E2M1 code is kept
+                            exp2_code_x2(w0, w1, f[i], f[i + 1]);
+                        } else {                     // FMA pipe: the value enters the row sum
                             exp2_fma_x2(w0, w1, f[i], f[i + 1]);
                         }
                     }
@@ -587,8 +609,10 @@ cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
     kp.nq2 = (a.N + C::kRows - 1) / C::kRows;
     kp.nkv = (a.N + T - 1) / T;
     kp.groups = (a.N + 127) / 128;
-    kp.p_thresh = a.p_thresh;
     kp.kq = static_cast<float>(static_cast<double>(a.softmax_scale) * 1.4426950408889634);
+    kp.e_sign = a.qmax >= 8.f ? 1.f : -1.f;
+    kp.e_off = a.qmax >= 8.f ? 0.f : static_cast<float>(std::log2(static_cast<double>(a.qmax)));
+    kp.e_add = a.qmax >= 8.f ? -2 : 0;
     dim3 grid(static_cast<unsigned>(a.BH * kp.nq2));
     mxattn_fwd_kernel<D, T, PNQ><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, kp);
     return cudaGetLastError();

@@ -40,7 +40,7 @@ struct AttnArgs {
     int d;
     int kv_tile;
     int pnq;
-    uint32_t p_thresh;  // block-exponent mantissa threshold for P (fp32 bits)
+    float qmax;         // scale boundary of P's block exponents, in (4, 8] (8 = OCP)
     float softmax_scale;
 };
 

@@ -377,6 +377,45 @@ __device__ __forceinline__ void exp2_fma_x2(float w0, float w1, float& v0, float
     v1 = __uint_as_float(p1 + (t1 << 23));
 }
 
+// A stand-in for 2^w whose E2M1 code (cvt.rn.satfinite.e2m1x2) equals the
+// code of 2^w, for two values on the FMA pipe.  The code of 2^w depends only
+// on where w falls against the E2M1 rounding points: the integer part
+// n = floor(w) picks the binade and the fraction f = w - n decides the
+// mantissa, whose rounding points 1.25, 1.5 and 1.75 are crossed at
+// f = log2(1.25), log2(1.5), log2(1.75).  z(f) = 1 + f (c1 + f (c2 + f c3))
+// is the cubic that passes through those three points and z(0) = 1 exactly
+// (coefficients from csrc/exp2_code_fit.py), is increasing on [0, 1) and stays
+// below 2, so 2^n * z(f) falls on the same side of every rounding point as
+// 2^w (up to fp32 rounding, a few ulp of f, as for ex2.approx).  Its value is
+// NOT 2^w (up to 7.7e-4 off between the points): use it only where nothing
+// but the code is kept.  Inputs are clamped at -8 (every w < -2 has code 0)
+// so the exponent field stays normal.
+__device__ __forceinline__ void exp2_code_x2(float w0, float w1, float& v0, float& v1) {
+    w0 = fmaxf(w0, -8.f);
+    w1 = fmaxf(w1, -8.f);
+    uint32_t p0, p1, t0, t1;
+    asm("{\n\t.reg .b64 w, t, n, f, p, c;\n\t"
+        "mov.b64 w, {%4, %5};\n\t"
+        "mov.b64 c, {%6, %6};\n\t"
+        "add.rm.f32x2 t, w, c;\n\t"      // floor(w) lands in the low mantissa bits of t
+        "sub.rn.f32x2 n, t, c;\n\t"      // n = floor(w)
+        "sub.rn.f32x2 f, w, n;\n\t"      // f in [0, 1]
+        "mov.b64 p, {%10, %10};\n\t"
+        "mov.b64 c, {%9, %9};\n\t"
+        "fma.rn.f32x2 p, p, f, c;\n\t"
+        "mov.b64 c, {%8, %8};\n\t"
+        "fma.rn.f32x2 p, p, f, c;\n\t"
+        "mov.b64 c, {%7, %7};\n\t"
+        "fma.rn.f32x2 p, p, f, c;\n\t"
+        "mov.b64 {%0, %1}, p;\n\t"
+        "mov.b64 {%2, %3}, t;\n\t}"
+        : "=r"(p0), "=r"(p1), "=r"(t0), "=r"(t1)
+        : "f"(w0), "f"(w1), "f"(12582912.0f),  // 1.5 * 2^23
+          "f"(1.0f), "f"(0x1.63d846p-1f), "f"(0x1.d566bep-3f), "f"(0x1.334fcep-4f));
+    v0 = __uint_as_float(p0 + (t0 << 23));
+    v1 = __uint_as_float(p1 + (t1 << 23));
+}
+
 // ------------------------------------------------------------------ E2M1 / E8M0 helpers
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -401,21 +440,12 @@ __device__ __forceinline__ uint32_t pack_e2m1x8(const float (&x)[8]) {
     return out;
 }
 
-// Block exponent from the fp32 bit pattern of the block maximum (>= 0) under
-// a scale boundary Qmax in (4, 8]: the smallest e with amax <= Qmax * 2^e is
-// floor(log2 amax) - 2, plus one when the significand exceeds Qmax / 4, i.e.
-// when the mantissa field exceeds `mant_thresh` = floor((Qmax/4 - 1) * 2^23).
-//   UOS (Qmax = 7.25): 0x680000.   OCP (floor(log2 amax) - 2): 0x7FFFFF, never
-//   exceeded.  Zero and subnormal maxima give -127.
-__device__ __forceinline__ int block_exponent_f32(uint32_t amax_bits, uint32_t mant_thresh) {
-    const int E = static_cast<int>((amax_bits >> 23) & 0xFFu);
-    if (E == 0) return -127;
-    int e = E - 129 + (((amax_bits & 0x7FFFFFu) > mant_thresh) ? 1 : 0);
-    return e < -127 ? -127 : (e > 127 ? 127 : e);
-}
-
-// Same rule on a bfloat16 bit pattern: mantissa field > floor((Qmax/4 - 1) * 2^7)
-// (UOS: 0x68; OCP: 0x7F, never exceeded).
+// Block exponent from the bfloat16 bit pattern of a block maximum (>= 0)
+// under a scale boundary Qmax in (4, 8]: the smallest e with amax <= Qmax * 2^e
+// is floor(log2 amax) - 2, plus one when the significand exceeds Qmax / 4,
+// i.e. when the mantissa field exceeds floor((Qmax/4 - 1) * 2^7) (UOS: 0x68;
+// OCP, floor(log2 amax) - 2: 0x7F, never exceeded).  Zero and subnormal
+// maxima give -127.
 __device__ __forceinline__ int block_exponent_bf16(uint32_t amax_bits, uint32_t mant_thresh) {
     const int E = static_cast<int>((amax_bits >> 7) & 0xFFu);
     if (E == 0) return -127;
