@@ -227,9 +227,10 @@ def quantize_sweep_point(torch, mx, peaks, peak_kind, log2n=30, iters=10):
     return out
 
 
-# Exponentials per S element in mxattn_fwd_kernel: three of every four pairs on
-# the MUFU (ex2.approx), one on the FMA pipe; plus one per 32-column block.
-MUFU_EX2_PER_ELEMENT = 0.75 + 1.0 / 32
+# MUFU exponentials per S element in mxattn_fwd_kernel with PNQ: 9 of every 16
+# pairs on the MUFU (ex2.approx), 7 on the FMA pipe; plus the rescale factor,
+# one per row and 128-column key tile.  Block exponents take no exponential.
+MUFU_EX2_PER_ELEMENT = 9.0 / 16 + 1.0 / 128
 
 
 def mufu_roofline(w, attn_ms, clocks, sms=148, ex2_per_clk_per_sm=16):
