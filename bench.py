@@ -269,6 +269,53 @@ def selected_workload(args):
     return w
 
 
+QMAX_STUDY = (6.0, 6.5, 7.0, 7.25, 7.5, 7.75, 8.0)
+
+
+def qmax_study(args):
+    """Scale-boundary study: O error against exact attention (fp64, unquantized
+    bf16 inputs) for boundaries Qmax in [6, 8] (8 = OCP), PNQ on and off, on
+    four input distributions.  The error is the relative Frobenius norm over a
+    seeded sample of query rows per head (all heads)."""
+    import torch
+
+    from mxfp4_microscaled_quantization_b200 import mxattn as mx
+
+    torch.cuda.set_device(0)
+    vid = wl.WORKLOADS["video_dit"]
+    cases = [
+        ("gaussian", wl.gaussian_qkv(1, 8, 4096, 128, seed=0)),
+        ("student_t3", wl.student_t_qkv(1, 8, 4096, 128, seed=0)),
+        ("outlier", wl.outlier_qkv(1, 8, 4096, 128, seed=0)),
+        ("video_dit_4heads", wl.video_dit_qkv(1, 4, vid.frames, vid.rows, vid.cols, vid.d, seed=0)),
+    ]
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)  # noqa: E731
+    out_rows = []
+    for name, (Q, K, V) in cases:
+        q, k, v = to_dev(Q), to_dev(K), to_dev(V)
+        B, H, N, d = q.shape
+        rows = torch.from_numpy(np.sort(np.random.default_rng(7).choice(N, min(N, 512), replace=False))).cuda()
+        qd, kd, vd = q.double(), k.double(), v.double()
+        s = torch.einsum("bhrd,bhnd->bhrn", qd[:, :, rows], kd) / math.sqrt(d)
+        exact = torch.einsum("bhrn,bhnd->bhrd", torch.softmax(s, dim=-1), vd)
+        ws = mx.new_workspace(B, H, N, d)
+        for qmax in QMAX_STUDY:
+            for pnq in (True, False):
+                o = mx.mxattn_forward(q, k, v, 128, pnq, qmax, workspace=ws)
+                torch.cuda.synchronize()
+                if mx.mxattn_workspace_status(ws) != 0:
+                    raise RuntimeError("attention kernel reported a timeout")
+                got = o[:, :, rows].double()
+                rel = float((got - exact).norm() / exact.norm())
+                out_rows.append({"inputs": name, "qmax": qmax, "pnq": pnq, "rel_err": rel})
+    line = {"study": "scale boundary Qmax vs O error against exact fp64 attention",
+            "shapes": "gaussian / student_t3 / outlier: B=1 H=8 N=4096 d=128; video_dit_4heads: B=1 H=4 "
+                      "N=32760 d=128; kv_tile 128; 512 seeded query rows per head",
+            "rows": out_rows}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_gpu(args, rank, world, local_rank):
     import torch
 
@@ -426,6 +473,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(wl.WORKLOADS), default="video_dit",
                     help="workload to time (default: the video-DiT configuration the metric is quoted on)")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller cases for profiling)")
+    ap.add_argument("--qmax-study", action="store_true",
+                    help="instead of the timed step: O error against exact attention over scale boundaries in [6, 8]")
     ap.add_argument("--quick", action="store_true",
                     help="timed steps only: no CPU baseline, no end-to-end leg, no quantize sweep")
     args = ap.parse_args()
@@ -435,6 +484,8 @@ def main():
     args.warmup = max(args.warmup, 3)  # timing rule: at least 3 warm-up steps
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.qmax_study:
+        return qmax_study(args) if rank == 0 else 0
     return run_gpu(args, rank, world, local_rank)
 
 

@@ -29,6 +29,7 @@ __all__ = [
     "outlier_qkv",
     "video_dit_qkv",
     "student_t_matrix",
+    "student_t_qkv",
     "make_qkv",
 ]
 
@@ -151,6 +152,15 @@ def student_t_matrix(n_elems, cols=4096, seed=0, nu=3.0, scale=0.5):
         x = rng.standard_t(nu, size=(r1 - r0, cols)).astype(np.float32) * np.float32(scale)
         out[r0:r1] = f32_to_bf16_bits(x)
     return out
+
+
+def student_t_qkv(B, H, N, d, seed=0, nu=3.0):
+    """Heavy-tailed inputs: Q, K, V drawn i.i.d. StudentT(nu), nu = 3 by default."""
+    out = []
+    for t in range(3):
+        rng = np.random.default_rng(seed + t)
+        out.append(f32_to_bf16_bits(rng.standard_t(nu, size=(B, H, N, d)).astype(np.float32)))
+    return tuple(out)
 
 
 def make_qkv(w: Workload, seed=0):
