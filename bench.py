@@ -260,6 +260,14 @@ def rank_seed(rank: int) -> int:
     return rank
 
 
+def head_range(H: int, rank: int, world: int):
+    """Heads [lo, hi) of one problem that rank `rank` computes when the heads are
+    sharded over `world` ranks: contiguous, sizes differing by at most one."""
+    base, extra = divmod(H, world)
+    lo = rank * base + min(rank, extra)
+    return lo, lo + base + (1 if rank < extra else 0)
+
+
 def selected_workload(args):
     w = wl.WORKLOADS[args.workload]
     if args.heads:
@@ -329,11 +337,23 @@ def run_gpu(args, rank, world, local_rank):
         import torch.distributed as dist
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    w = selected_workload(args)
+    w_full = selected_workload(args)
     peaks, peak_kind = load_peaks()
-    B, H, N, d = w.B, w.H, w.N, w.d
+    if args.shard == "heads":
+        # One problem, its heads split over the ranks (no exchange: heads are independent).
+        import dataclasses
 
-    Q, K, V = wl.make_qkv(w, seed=rank_seed(rank))
+        lo, hi = head_range(w_full.H, rank, world)
+        if hi <= lo:
+            raise ValueError(f"{w_full.H} heads cannot be sharded over {world} ranks")
+        Q, K, V = (np.ascontiguousarray(a[:, lo:hi]) for a in wl.make_qkv(w_full, seed=0))
+        w = dataclasses.replace(w_full, H=hi - lo)
+    else:
+        w = w_full
+        Q, K, V = wl.make_qkv(w, seed=rank_seed(rank))
+    B, H, N, d = w.B, w.H, w.N, w.d
+    # whole-job work per step: every rank's problem (replicas) or the one sharded problem
+    job_flops = w_full.flops if args.shard == "heads" else world * w.flops
     base = None
     if rank == 0 and not args.quick:
         base = cpu_baseline(Q, K, V, w, budget_s=args.cpu_budget)
@@ -376,7 +396,7 @@ def run_gpu(args, rank, world, local_rank):
         raise RuntimeError("attention kernel reported a timeout")
     total_ms, attn_avg_ms = max_over_ranks([total_ms, sum(attn_ms) / len(attn_ms)], dist, "cuda")
     ms_per_step = total_ms / args.steps
-    value = world * w.flops / (ms_per_step / 1e3) / 1e12
+    value = job_flops / (ms_per_step / 1e3) / 1e12
 
     e2e_ms = None
     if not args.quick:
@@ -410,9 +430,12 @@ def run_gpu(args, rank, world, local_rank):
         clocks = clk.summary()
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "strong" if args.shard == "heads" else "weak",
             "vs_baseline": None, "dtype": "mxfp4 (e2m1 x e8m0, fp32 accumulate)", "data": "synthetic",
-            "config": {**config_dict(w), "parallelism": f"{world} independent replicas (one batch per rank)"},
+            "config": {**config_dict(w_full), "parallelism": (
+                f"heads sharded over {world} ranks (one problem, no exchange)" if args.shard == "heads"
+                else f"{world} independent replicas (one batch per rank)")},
             "pct_of_fp4_peak": 100.0 * value / world / peak,
             "roofline": {"bound": "tensor", "kernel": f"mxattn_fwd_kernel<{w.d},{w.kv_tile}>", "achieved": attn_tflops,
                          "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
@@ -423,7 +446,7 @@ def run_gpu(args, rank, world, local_rank):
                          "frac_of_9pf_spec": attn_tflops / 9000.0},
             "cpu_baseline": base,
             "e2e": None if e2e_ms is None else {
-                "value": world * w.flops / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+                "value": job_flops / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": 3 * B * H * N * d * 2, "d2h_bytes_per_step": B * H * N * d * 4,
                 "ms_per_step": e2e_ms, "api": "attention_from_host -> mxattn_forward"},
             "mufu_roofline": mufu_roofline(w, attn_avg_ms, clocks),
@@ -473,6 +496,9 @@ def main():
     ap.add_argument("--workload", choices=sorted(wl.WORKLOADS), default="video_dit",
                     help="workload to time (default: the video-DiT configuration the metric is quoted on)")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller cases for profiling)")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="N > 1: one independent batch per rank (weak scaling, default) or the heads of one "
+                         "problem split over the ranks (strong scaling)")
     ap.add_argument("--qmax-study", action="store_true",
                     help="instead of the timed step: O error against exact attention over scale boundaries in [6, 8]")
     ap.add_argument("--quick", action="store_true",
