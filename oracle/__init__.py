@@ -11,7 +11,9 @@ Data-Free Optimal Scaling and Pre-Normalization Quantization for MXFP4
 Attention").  Every function here is pinned by the ``-m "not gpu"`` tests
 (E2M1 grid and brute-force rounding, the OCP and UOS scale invariants,
 equivariance, exact online softmax, PNQ normalization, hand-derived golden
-cases); none is "parity unpinned".
+cases; for the NVFP4 comparison variant, torch's float8_e4m3fn conversion,
+brute-force element rounding, equivariance and special cases); none is
+"parity unpinned".
 """
 from __future__ import annotations
 
@@ -69,6 +71,19 @@ def lib():
         L.oracle_max_threads.restype = ctypes.c_int
         L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
         L.oracle_e2m1_decode.restype = ctypes.c_double
+        L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_decode.restype = ctypes.c_double
+        L.oracle_e4m3_encode_batch.argtypes = [P, i64, P]
+        L.oracle_nvfp4_global.argtypes = [ctypes.c_double]
+        L.oracle_nvfp4_global.restype = ctypes.c_float
+        L.oracle_bf16_amax.argtypes = [P, i64]
+        L.oracle_bf16_amax.restype = ctypes.c_double
+        L.oracle_nvfp4_quantize_rows.argtypes = [P, i64, i64, ctypes.c_float, P, P]
+        L.oracle_nvfp4_quantize_cols.argtypes = [P, i64, i64, i64, P, P, P]
+        L.oracle_nvfp4_dequantize_rows.argtypes = [P, P, i64, i64, ctypes.c_float, P]
+        L.oracle_nvfp4_attention_head.argtypes = [P, P, P, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_double, P, i64, P, ctypes.c_int]
+        L.oracle_nvfp4_attention_head.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -199,5 +214,108 @@ def attention(Q, K, V, kv_tile, rule="uos", pnq=True, p_rule=None, scale=None, r
                                            _ptr(o), int(nthreads))
         if st != 0:
             raise RuntimeError(f"oracle_attention_head failed with status {st}")
+        ov[bh] = o
+    return out
+
+
+# ---------------------------------------------------------------- NVFP4 comparison variant
+# Definitions and readings beside the C code (oracle.c, "NVFP4 comparison variant").
+
+def e4m3_decode(codes) -> np.ndarray:
+    codes = np.asarray(codes, dtype=np.uint8)
+    return np.array([lib().oracle_e4m3_decode(int(c)) for c in codes.ravel()]).reshape(codes.shape)
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """|v| -> E4M3 code, round to nearest even, saturating at 448."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e4m3_encode_batch(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def nvfp4_global(amax) -> np.float32:
+    """Second-level scale g = 448 / amax (fp32) of a slice with absolute maximum amax."""
+    return np.float32(lib().oracle_nvfp4_global(float(amax)))
+
+
+def nvfp4_head_globals(x_bits: np.ndarray) -> np.ndarray:
+    """bf16 bits [B, H, N, d] -> g per (batch, head), float32 [B, H]."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    B, H = x.shape[:2]
+    flat = x.reshape(B * H, -1)
+    g = [nvfp4_global(lib().oracle_bf16_amax(_ptr(np.ascontiguousarray(flat[i])), flat.shape[1]))
+         for i in range(B * H)]
+    return np.array(g, dtype=np.float32).reshape(B, H)
+
+
+def nvfp4_quantize_rows(x_bits: np.ndarray, g):
+    """bf16 bits [rows, cols] (cols % 16 == 0), one scale g -> (codes [rows, cols/2], E4M3 scales [rows, cols/16])."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    cols = x.shape[-1]
+    assert cols % 16 == 0
+    rows = x.size // cols
+    codes = np.empty(x.shape[:-1] + (cols // 2,), dtype=np.uint8)
+    scales = np.empty(x.shape[:-1] + (cols // 16,), dtype=np.uint8)
+    lib().oracle_nvfp4_quantize_rows(_ptr(x), rows, cols, float(g), _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def nvfp4_quantize_cols(v_bits: np.ndarray, g):
+    """V bf16 bits [BH..., N, d], g one scale per (b, h) -> V^T (codes [..., d, Npad/2], scales [..., d, Npad/16])."""
+    v = np.ascontiguousarray(v_bits, dtype=np.uint16)
+    N, d = v.shape[-2:]
+    BH = v.size // (N * d)
+    npad = (N + 31) // 32 * 32
+    lead = v.shape[:-2]
+    gg = np.ascontiguousarray(np.broadcast_to(np.asarray(g, dtype=np.float32).ravel(), (BH,)))
+    codes = np.empty(lead + (d, npad // 2), dtype=np.uint8)
+    scales = np.empty(lead + (d, npad // 16), dtype=np.uint8)
+    lib().oracle_nvfp4_quantize_cols(_ptr(v), BH, N, d, _ptr(gg), _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def nvfp4_dequantize_rows(codes: np.ndarray, scales: np.ndarray, g) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    cols = codes.shape[-1] * 2
+    rows = codes.size * 2 // cols
+    out = np.empty(codes.shape[:-1] + (cols,), dtype=np.float64)
+    lib().oracle_nvfp4_dequantize_rows(_ptr(codes), _ptr(scales), rows, cols, float(g), _ptr(out))
+    return out
+
+
+def nvfp4_attention(Q, K, V, kv_tile, pnq=True, quant=True, p_quant=True, scale=None, rows=None, nthreads=0):
+    """NVFP4 attention forward on the CPU (fp64 loop, fp32 scale arithmetic).
+
+    Q, K, V: bf16 bits [B, H, N, d].  quant=False keeps every operand exact;
+    p_quant=False keeps only P exact.  rows as in `attention`.  Returns fp64 [B, H, R, d].
+    """
+    Q = np.ascontiguousarray(Q, dtype=np.uint16)
+    K = np.ascontiguousarray(K, dtype=np.uint16)
+    V = np.ascontiguousarray(V, dtype=np.uint16)
+    B, H, N, d = Q.shape
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    per_head_rows = []
+    for bh in range(B * H):
+        if rows is None:
+            r = np.arange(N, dtype=np.int64)
+        elif isinstance(rows, (list, tuple)):
+            r = np.asarray(rows[bh], dtype=np.int64)
+        else:
+            r = np.asarray(rows, dtype=np.int64)
+        per_head_rows.append(np.ascontiguousarray(r))
+    R = len(per_head_rows[0])
+    out = np.empty((B, H, R, d), dtype=np.float64)
+    Qf, Kf, Vf = (a.reshape(B * H, N, d) for a in (Q, K, V))
+    ov = out.reshape(B * H, R, d)
+    for bh in range(B * H):
+        o = np.empty((R, d), dtype=np.float64)
+        st = lib().oracle_nvfp4_attention_head(_ptr(Qf[bh]), _ptr(Kf[bh]), _ptr(Vf[bh]), N, d, kv_tile,
+                                               1 if quant else 0, 1 if p_quant else 0, 1 if pnq else 0,
+                                               float(scale), _ptr(per_head_rows[bh]), R, _ptr(o), int(nthreads))
+        if st != 0:
+            raise RuntimeError(f"oracle_nvfp4_attention_head failed with status {st}")
         ov[bh] = o
     return out
