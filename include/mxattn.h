@@ -231,6 +231,75 @@ mxattn_status mxattn_workspace_status(const void* workspace, mxattn_stream_t str
  */
 mxattn_status mxattn_wait_selftest(int arrive, unsigned timeout_us, unsigned* out, mxattn_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * NVFP4 comparison variant.  The abstract measures MXAttention against
+ * "NVFP4-based baselines" without defining them; this library's reading is
+ * NVIDIA's NVFP4 applied to the same four operands and the same softmax loop:
+ *   - E2M1 elements (as above) in blocks of 16 along the contraction axis,
+ *     one unsigned E4M3 (OCP FP8 E4M3) scale per block, and one fp32
+ *     second-level scale per (batch, head) slice of Q, K or V;
+ *   - g = 448 / max(amax_slice, 2^-100), block scale sb = E4M3(amax_block * g)
+ *     (round to nearest even, saturating at 448), element code
+ *     E2M1(x * ((6 g) / sb)), all in fp32 with round to nearest; a block whose
+ *     scale rounds to 0 holds zeros (sign kept); value = code * sb / (6 g);
+ *   - P (<= 1 by construction) uses g = 448 with blocks of 16 keys aligned to
+ *     key-tile starts; PNQ on/off as for MXFP4.
+ * Codes and scales decided from bf16 inputs are exact functions of these
+ * definitions (no approximation): the oracle reproduces them bit for bit.
+ * The tensor-core step is tcgen05.mma kind::mxf4nvf4 (block16, E4M3 scales).
+ * ------------------------------------------------------------------------- */
+
+/*
+ * Standalone NVFP4 quantization of a whole tensor (one second-level scale):
+ *   x:      bf16 [rows, cols], cols % 16 == 0, 16-byte aligned.
+ *   codes:  u8 [rows, cols/2] (4-byte aligned).  scales: u8 [rows, cols/16] E4M3.
+ *   gs:     device float[2], 4-byte aligned, written by the call: gs[0] = amax
+ *           of x, gs[1] = g = 448 / max(amax, 2^-100).
+ * Launches an amax pass, the quantizer and a one-thread kernel that stores g;
+ * rows == 0 launches nothing and returns MXATTN_OK.
+ * Errors: MXATTN_ERR_INVALID (null, misaligned, rows < 0, cols not a positive
+ * multiple of 16), MXATTN_ERR_CUDA (launch failed).
+ */
+mxattn_status mxattn_nvfp4_quantize(const void* x, int64_t rows, int64_t cols, uint8_t* codes, uint8_t* scales,
+                                    float* gs, mxattn_stream_t stream);
+
+/*
+ * Workspace bytes for the NVFP4 forward (0 for invalid shapes).  Regions, each
+ * on a 256-byte boundary, in order (G = ceil(N/128), Npad = ceil(N/32)*32):
+ *   status 256 bytes (u32 error word, as for the MXFP4 workspace)
+ *   q_codes B*H*N*d/2   k_codes B*H*N*d/2   vt_codes B*H*d*Npad/2
+ *   q_sf    B*H*G*(d/64)*512   k_sf B*H*G*(d/64)*512   vt_sf B*H*G*1024
+ *   amax    3*B*H u32 (fp32 bits of |Q|, |K|, |V| maxima per (b, h))
+ *   g       3*B*H fp32 (second-level scales of Q, K, V per (b, h))
+ * Scale regions are regrouped per 128 rows (Q, K) or 128 tokens (V^T) and
+ * per 64 columns of the contraction axis: 512-byte atoms in which row m (or
+ * channel m) and 16-element block b of the 64 columns sit at byte
+ * (m%32)*16 + (m/32)*4 + b; rows past N hold 0, unused V^T channel rows 0x38
+ * (E4M3 1.0).
+ */
+size_t mxattn_nvfp4_workspace_size(int B, int H, int N, int d);
+
+/*
+ * NVFP4 attention forward (non-causal), the same tile-ordered online softmax
+ * as mxattn_forward with every operand in NVFP4:
+ *   Q, K, V: bf16 [B, H, N, d], 16-byte aligned.  O: fp32 [B, H, N, d].
+ *   d in {64, 128}; kv_tile in {64, 128}; 1 <= N <= 2^24; B*H <= 65535;
+ *   pnq in {0, 1}; softmax_scale <= 0 selects 1/sqrt(d).
+ *   workspace: >= mxattn_nvfp4_workspace_size(B, H, N, d) bytes, 256-byte aligned.
+ * mxattn_nvfp4_prepare launches the amax pass and the Q/K and V^T quantizers
+ * into the workspace; mxattn_nvfp4_attend runs the attention kernel on it;
+ * mxattn_nvfp4_forward is the two in order.  The status word and
+ * mxattn_workspace_status work as for the MXFP4 workspace.
+ * Errors as mxattn_forward.
+ */
+mxattn_status mxattn_nvfp4_forward(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                   int kv_tile, int pnq, float softmax_scale, float* O, void* workspace,
+                                   size_t workspace_bytes, mxattn_stream_t stream);
+mxattn_status mxattn_nvfp4_prepare(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                   void* workspace, size_t workspace_bytes, mxattn_stream_t stream);
+mxattn_status mxattn_nvfp4_attend(int B, int H, int N, int d, int kv_tile, int pnq, float softmax_scale, float* O,
+                                  void* workspace, size_t workspace_bytes, mxattn_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* mxattn_status_string(mxattn_status status);
 

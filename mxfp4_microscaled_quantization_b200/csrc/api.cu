@@ -282,3 +282,132 @@ MXATTN_API mxattn_status mxattn_workspace_status(const void* workspace, mxattn_s
     if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MXATTN_ERR_CUDA;
     return (word & 4u) ? MXATTN_ERR_TIMEOUT : MXATTN_OK;
 }
+
+// ------------------------------------------------------------------ NVFP4 comparison variant
+
+namespace {
+
+struct NvLayout {
+    size_t status, q_codes, k_codes, vt_codes, q_sf, k_sf, v_sf, amax, gs, total;
+};
+
+bool make_layout_nv(int B, int H, int N, int d, NvLayout* L) {
+    if (B < 1 || H < 1 || N < 1 || N > kMaxN || (d != 64 && d != 128)) return false;
+    const size_t BH = static_cast<size_t>(B) * H;
+    const size_t G = (static_cast<size_t>(N) + 127) / 128;
+    const size_t npad = (static_cast<size_t>(N) + 31) / 32 * 32;
+    size_t off = 0;
+    L->status = off;
+    off += 256;
+    L->q_codes = off;
+    off = align256(off + BH * N * d / 2);
+    L->k_codes = off;
+    off = align256(off + BH * N * d / 2);
+    L->vt_codes = off;
+    off = align256(off + BH * d * npad / 2);
+    L->q_sf = off;
+    off = align256(off + BH * G * (d / 64) * 512);
+    L->k_sf = off;
+    off = align256(off + BH * G * (d / 64) * 512);
+    L->v_sf = off;
+    off = align256(off + BH * G * 1024);
+    L->amax = off;
+    off = align256(off + 3 * BH * 4);
+    L->gs = off;
+    off = align256(off + 3 * BH * 4);
+    L->total = off;
+    return true;
+}
+
+mxattn_status check_nv_args(int B, int H, int N, int d, int kv_tile, int pnq, const float* O, const void* ws,
+                            size_t ws_bytes, NvLayout* L) {
+    if (B < 1 || H < 1 || N < 1 || O == nullptr || ws == nullptr) return MXATTN_ERR_INVALID;
+    if (pnq != 0 && pnq != 1) return MXATTN_ERR_INVALID;
+    if (d != 64 && d != 128) return MXATTN_ERR_UNSUPPORTED;
+    if (kv_tile != 64 && kv_tile != 128) return MXATTN_ERR_UNSUPPORTED;
+    if (N > kMaxN || static_cast<int64_t>(B) * H > 65535) return MXATTN_ERR_UNSUPPORTED;
+    if (!make_layout_nv(B, H, N, d, L)) return MXATTN_ERR_INVALID;
+    if (ws_bytes < L->total || !aligned(ws, 256) || !aligned(O, 16)) return MXATTN_ERR_INVALID;
+    return MXATTN_OK;
+}
+
+}  // namespace
+
+MXATTN_API size_t mxattn_nvfp4_workspace_size(int B, int H, int N, int d) {
+    NvLayout L;
+    return make_layout_nv(B, H, N, d, &L) ? L.total : 0;
+}
+
+MXATTN_API mxattn_status mxattn_nvfp4_quantize(const void* x, int64_t rows, int64_t cols, uint8_t* codes,
+                                               uint8_t* scales, float* gs, mxattn_stream_t stream) {
+    if (rows < 0 || cols <= 0 || cols % 16 != 0) return MXATTN_ERR_INVALID;
+    if (rows == 0) return MXATTN_OK;  // nothing to do
+    if (x == nullptr || codes == nullptr || scales == nullptr || gs == nullptr) return MXATTN_ERR_INVALID;
+    if (!aligned(x, 16) || !aligned(codes, 4) || !aligned(gs, 4)) return MXATTN_ERR_INVALID;
+    cudaError_t e = mxattn::launch_nv_quantize_rows(x, rows, cols, codes, scales, gs,
+                                                     reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
+}
+
+MXATTN_API mxattn_status mxattn_nvfp4_prepare(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                              void* workspace, size_t workspace_bytes, mxattn_stream_t stream) {
+    NvLayout L;
+    float dummy_out[4];
+    mxattn_status st = check_nv_args(B, H, N, d, 128, 1, dummy_out, workspace, workspace_bytes, &L);
+    if (st != MXATTN_OK) return st;
+    if (Q == nullptr || K == nullptr || V == nullptr) return MXATTN_ERR_INVALID;
+    if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16)) return MXATTN_ERR_INVALID;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const int64_t BH = static_cast<int64_t>(B) * H;
+    const int G = (N + 127) / 128;
+    uint32_t* amax = reinterpret_cast<uint32_t*>(ws + L.amax);
+    float* gs = reinterpret_cast<float*>(ws + L.gs);
+    cudaError_t e = mxattn::launch_nv_amax(Q, K, V, 3, static_cast<int64_t>(N) * d, BH, amax, s);
+    if (e != cudaSuccess) return MXATTN_ERR_CUDA;
+    e = mxattn::launch_nv_quantize_qk(Q, K, ws + L.q_codes, ws + L.k_codes, ws + L.q_sf, ws + L.k_sf, amax, amax + BH,
+                                      gs, gs + BH, BH, N, d, G, reinterpret_cast<uint32_t*>(ws + L.status), s);
+    if (e != cudaSuccess) return MXATTN_ERR_CUDA;
+    e = mxattn::launch_nv_quantize_vt(V, BH, N, d, G, amax + 2 * BH, gs + 2 * BH, ws + L.vt_codes, ws + L.v_sf, s);
+    return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
+}
+
+MXATTN_API mxattn_status mxattn_nvfp4_attend(int B, int H, int N, int d, int kv_tile, int pnq, float softmax_scale,
+                                             float* O, void* workspace, size_t workspace_bytes,
+                                             mxattn_stream_t stream) {
+    NvLayout L;
+    mxattn_status st = check_nv_args(B, H, N, d, kv_tile, pnq, O, workspace, workspace_bytes, &L);
+    if (st != MXATTN_OK) return st;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    mxattn::AttnArgs a{};
+    a.q_codes = ws + L.q_codes;
+    a.k_codes = ws + L.k_codes;
+    a.vt_codes = ws + L.vt_codes;
+    a.q_sf = ws + L.q_sf;
+    a.k_sf = ws + L.k_sf;
+    a.v_sf = ws + L.v_sf;
+    a.O = O;
+    a.status = reinterpret_cast<uint32_t*>(ws + L.status);
+    a.BH = static_cast<int64_t>(B) * H;
+    a.N = N;
+    a.d = d;
+    a.kv_tile = kv_tile;
+    a.pnq = pnq;
+    a.qmax = 8.f;  // unused by the NVFP4 path
+    a.softmax_scale = resolve_scale(softmax_scale, d);
+    a.nv = 1;
+    a.gs = reinterpret_cast<const float*>(ws + L.gs);
+    cudaError_t e = mxattn::launch_attention(a, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
+}
+
+MXATTN_API mxattn_status mxattn_nvfp4_forward(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                              int kv_tile, int pnq, float softmax_scale, float* O, void* workspace,
+                                              size_t workspace_bytes, mxattn_stream_t stream) {
+    NvLayout L;
+    mxattn_status st = check_nv_args(B, H, N, d, kv_tile, pnq, O, workspace, workspace_bytes, &L);
+    if (st != MXATTN_OK) return st;
+    st = mxattn_nvfp4_prepare(Q, K, V, B, H, N, d, workspace, workspace_bytes, stream);
+    if (st != MXATTN_OK) return st;
+    return mxattn_nvfp4_attend(B, H, N, d, kv_tile, pnq, softmax_scale, O, workspace, workspace_bytes, stream);
+}

@@ -56,7 +56,7 @@ constexpr uint32_t kTimeoutCode = 4u;           // MXATTN_ERR_TIMEOUT
 // Suspend hint for the producer's and the MMA issuer's waits (0: plain try_wait).
 constexpr uint32_t kRoleWaitHintNs = MXATTN_ROLE_WAIT_HINT_NS;
 
-template <int D, int T>
+template <int D, int T, bool NV = false>
 struct Cfg {
     static constexpr int kStages = 4;
     static constexpr int kTiles = 2;                  // query tiles per CTA
@@ -80,7 +80,19 @@ struct Cfg {
     static constexpr int kVLoadBytes = D * T / 2;
     static constexpr int kVStride = ((kVRows * T / 2) + 1023) / 1024 * 1024;
     static constexpr int kPBytes = 128 * T / 2;
-    static constexpr int kSfBytes = 512;
+    // Scale factors travel in 512-byte atoms (128 rows x 4 scale bytes, the
+    // order tcgen05 reads them).  MXFP4 (block 32): one atom covers a 128-row
+    // tile for any d or kv_tile here.  NVFP4 (block 16): one atom per 64
+    // columns of the contraction axis.
+    static constexpr int kQAtoms = NV ? D / 64 : 1;                       // Q and K, per 128-row group
+    static constexpr int kVAtoms = NV ? T / 64 : 1;                       // V^T per key tile; P per tile
+    static constexpr int kQsfBytes = 512 * kQAtoms;
+    static constexpr int kVsfGroupBytes = NV ? 1024 : 512;               // V^T scales per 128 tokens in HBM
+    static constexpr int kVsfBytes = 512 * kVAtoms;                      // V^T scales loaded per key tile
+    static constexpr int kPsfBytes = 512 * kVAtoms;
+    static constexpr int kSfBytes = 512;                                  // one atom
+    // TMEM slots for the K and V^T scale factors (NVFP4's larger scales leave room for two)
+    static constexpr int kSfSlots = NV ? 2 : kStages;
     static constexpr int kOCols = D + 16;
     // Of the 16 exponential pairs of a 32-column block, this many go to the FMA
     // pipe instead of the MUFU: 7 with PNQ (the code-only stand-in for 2^w,
@@ -102,10 +114,10 @@ struct Cfg {
     static constexpr int kOffV = kOffK + kStages * kKBytes;             // [kStages]
     static constexpr int kOffP = kOffV + kStages * kVStride;            // [kTiles]
     static constexpr int kOffQsf = kOffP + kTiles * kPBytes;            // [kTiles]
-    static constexpr int kOffKsf = kOffQsf + kTiles * kSfBytes;         // [kStages]
-    static constexpr int kOffVsf = kOffKsf + kStages * kSfBytes;        // [kStages]
-    static constexpr int kOffPsf = kOffVsf + kStages * kSfBytes;        // [kTiles]
-    static constexpr int kOffVsfConst = kOffPsf + kTiles * kSfBytes;
+    static constexpr int kOffKsf = kOffQsf + kTiles * kQsfBytes;        // [kStages]
+    static constexpr int kOffVsf = kOffKsf + kStages * kQsfBytes;       // [kStages]
+    static constexpr int kOffPsf = kOffVsf + kStages * kVsfBytes;       // [kTiles]
+    static constexpr int kOffVsfConst = kOffPsf + kTiles * kPsfBytes;
     static constexpr int kOffBar = kOffVsfConst + kSfBytes;
     // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S],
     //           s_full[kTiles], s_loaded[kTiles], p_full[kTiles], o_done[kTiles], drain
@@ -118,11 +130,12 @@ struct Cfg {
     // TMEM columns: one S buffer shared by both tiles, then O per tile, then scale factors
     static constexpr uint32_t kColS = 0;
     static constexpr uint32_t kColO = T;  // + t * kOCols
-    static constexpr uint32_t kColQsf = (T + kTiles * kOCols + 3) / 4 * 4;  // + 4 t
-    static constexpr uint32_t kColKsf = kColQsf + 4 * kTiles;               // + 4 s
-    static constexpr uint32_t kColPsf = kColKsf + 4 * kStages;              // + 4 t
-    static constexpr uint32_t kColVsf = kColPsf + 4 * kTiles;               // + 8 s
-    static constexpr uint32_t kColsUsed = kColVsf + 8 * kStages;
+    // (4 columns per atom; a V^T atom also has 4 columns for rows 128..255)
+    static constexpr uint32_t kColQsf = (T + kTiles * kOCols + 3) / 4 * 4;  // + 4 kQAtoms t
+    static constexpr uint32_t kColKsf = kColQsf + 4 * kQAtoms * kTiles;     // + 4 kQAtoms slot
+    static constexpr uint32_t kColPsf = kColKsf + 4 * kQAtoms * kSfSlots;   // + 4 kVAtoms t
+    static constexpr uint32_t kColVsf = kColPsf + 4 * kVAtoms * kTiles;     // + 8 kVAtoms slot
+    static constexpr uint32_t kColsUsed = kColVsf + 8 * kVAtoms * kSfSlots;
     static_assert(kColsUsed <= 512, "TMEM budget");
     static_assert(kSmemUsed + 1024 <= 227 * 1024, "shared memory budget");
 };
@@ -146,6 +159,9 @@ struct KParams {
     float e_sign;
     float e_off;
     int e_add;
+    // NVFP4: the second-level scales g of Q, K, V per (batch, head), [3][BH]
+    const float* gs;
+    int BH;
 };
 
 // Maximum of 32 values as a depth-4 tree of 3-input max instructions.
@@ -161,16 +177,23 @@ __device__ __forceinline__ float block_max32(const float* v) {
     return fmax3(u0, u1, fmaxf(u2, u3));
 }
 
+// Maximum of 16 values.
+__device__ __forceinline__ float block_max16(const float* v) {
+    const float t0 = fmax3(v[0], v[1], v[2]), t1 = fmax3(v[3], v[4], v[5]), t2 = fmax3(v[6], v[7], v[8]);
+    const float t3 = fmax3(v[9], v[10], v[11]), t4 = fmax3(v[12], v[13], v[14]);
+    return fmax3(fmax3(t0, t1, t2), t3, fmaxf(t4, v[15]));
+}
+
 __device__ __forceinline__ uint64_t sf_desc(const void* p) {
     // 32 rows x 16 bytes, rows contiguous: core matrices of 8 rows 128 bytes apart
     return smem_desc(smem_u32(p), 0, 128, kLayoutNone);
 }
 
-template <int D, int T, bool PNQ>
-__global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
+template <int D, int T, bool PNQ, bool NV>
+__global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
     mxattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const KParams p) {
-    using C = Cfg<D, T>;
+    using C = Cfg<D, T, NV>;
     constexpr int S = C::kStages;
     constexpr int NT = C::kTiles;
     extern __shared__ uint8_t smem_raw[];
@@ -201,7 +224,6 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
-    const int lane = tid & 31;
     const int bh = blockIdx.x / p.nq2;
     const int qp = blockIdx.x % p.nq2;  // pair index: rows [256 qp, 256 qp + 256)
     const int nkv = p.nkv;
@@ -231,8 +253,9 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
         const int row = D + w / (T / 8);
         reinterpret_cast<uint32_t*>(sV + s * C::kVStride + D * (T / 2))[w] = (row == D) ? 0x22222222u : 0u;
     }
-    // Scale factors of V^T rows 128..255 (only used when D = 128): all 2^0.
-    for (int idx = tid; idx < 128; idx += C::kThreads) reinterpret_cast<uint32_t*>(sVsfConst)[idx] = 0x7F7F7F7Fu;
+    // Scale factors of V^T rows 128..255 (only used when D = 128): all 1 (E8M0 2^0, or E4M3 1.0).
+    for (int idx = tid; idx < 128; idx += C::kThreads)
+        reinterpret_cast<uint32_t*>(sVsfConst)[idx] = NV ? 0x38383838u : 0x7F7F7F7Fu;
     fence_proxy_async_smem();
     if (warp == C::kMmaWarp) {
         tmem_alloc(tmem_holder, 512);
@@ -260,12 +283,13 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
         // ------------------------------------------------------------ TMA producer
             int k_issued = 0, v_issued = 0;
             if (leader) {
-                mbar_arrive_expect_tx(bar_q, NT * (C::kQBytes + C::kSfBytes));
+                mbar_arrive_expect_tx(bar_q, NT * (C::kQBytes + C::kQsfBytes));
                 for (int t = 0; t < NT; ++t) {
                     const int g = 2 * qp + t;  // 128-row group of tile t (may lie past N: zero-filled)
                     tma_load_3d(sQ + t * C::kQBytes, &tmQ, bar_q, 0, g * 128, bh);
                     const int gs = g < p.groups ? g : p.groups - 1;  // keep the scale copy inside the buffer
-                    bulk_load(sQsf + t * 512, p.q_sf + (static_cast<size_t>(bh) * p.groups + gs) * 512, 512, bar_q);
+                    bulk_load(sQsf + t * C::kQsfBytes, p.q_sf + (static_cast<size_t>(bh) * p.groups + gs) * C::kQsfBytes,
+                              C::kQsfBytes, bar_q);
                 }
             }
             __syncwarp();
@@ -275,17 +299,19 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                 const size_t grp = static_cast<size_t>(bh) * p.groups + (j * T) / 128;
                 if (j >= S && !wait(bar_k_empty + s, (n - 1) & 1)) break;
                 if (leader) {
-                    mbar_arrive_expect_tx(bar_k_full + s, C::kKBytes + C::kSfBytes);
+                    mbar_arrive_expect_tx(bar_k_full + s, C::kKBytes + C::kQsfBytes);
                     tma_load_3d(sK + s * C::kKBytes, &tmK, bar_k_full + s, 0, j * T, bh);
-                    bulk_load(sKsf + s * 512, p.k_sf + grp * 512, 512, bar_k_full + s);
+                    bulk_load(sKsf + s * C::kQsfBytes, p.k_sf + grp * C::kQsfBytes, C::kQsfBytes, bar_k_full + s);
                 }
                 __syncwarp();
                 k_issued = j + 1;
                 if (j >= S && !wait(bar_v_empty + s, (n - 1) & 1)) break;
                 if (leader) {
-                    mbar_arrive_expect_tx(bar_v_full + s, C::kVLoadBytes + C::kSfBytes);
+                    mbar_arrive_expect_tx(bar_v_full + s, C::kVLoadBytes + C::kVsfBytes);
                     tma_load_3d(sV + s * C::kVStride, &tmV, bar_v_full + s, j * (T / 2), 0, bh);
-                    bulk_load(sVsf + s * 512, p.v_sf + grp * 512, 512, bar_v_full + s);
+                    // NVFP4 with 64-key tiles: the key tile is one of the group's two 64-token atoms
+                    const size_t vsf_off = grp * C::kVsfGroupBytes + ((NV && T == 64) ? (j & 1) * 512 : 0);
+                    bulk_load(sVsf + s * C::kVsfBytes, p.v_sf + vsf_off, C::kVsfBytes, bar_v_full + s);
                 }
                 __syncwarp();
                 v_issued = j + 1;
@@ -316,17 +342,28 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
             auto issue_s = [&](int t, int j) -> bool {
                 const int s = j % S;
                 const uint32_t n = j / S;
+                const int slot = j % C::kSfSlots;
                 if (t == 0 && !wait(bar_k_full + s, n & 1)) return false;
                 tc_fence_after_sync();  // after the K wait, or after the wait for the S buffer to be read
                 const uint64_t qdesc = qdesc0 + static_cast<uint32_t>(t * (C::kQBytes >> 4));
                 const uint64_t kdesc = kdesc0 + static_cast<uint32_t>(s * (C::kKBytes >> 4));
-                const uint32_t ksf = tbase + C::kColKsf + 4 * s + ((T == 64) ? 2 * (j & 1) : 0);
+                const uint32_t ksf_col = tbase + C::kColKsf + 4 * C::kQAtoms * slot;
+                const uint32_t ksf = ksf_col + ((T == 64) ? 2 * (j & 1) : 0);  // rows 64..127 of the group: +2 columns
                 if (leader) {
-                    if (t == 0) tc_cp_sf(tbase + C::kColKsf + 4 * s, ksf0 + static_cast<uint32_t>(s * (512 >> 4)));
+                    if (t == 0) {
 #pragma unroll
-                    for (int kk = 0; kk < D / 64; ++kk)
-                        tc_mma_mxf4(t_s, qdesc + 2 * kk, kdesc + 2 * kk, mxf4_idesc(T, 2 * kk, 2 * kk),
-                                    tbase + C::kColQsf + 4 * t, ksf, kk > 0 ? 1u : 0u);
+                        for (int a = 0; a < C::kQAtoms; ++a)
+                            tc_cp_sf(ksf_col + 4 * a, ksf0 + static_cast<uint32_t>((s * C::kQsfBytes + 512 * a) >> 4));
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < D / 64; ++kk) {
+                        if constexpr (NV)
+                            tc_mma_nvf4(t_s, qdesc + 2 * kk, kdesc + 2 * kk, nvf4_idesc(T),
+                                        tbase + C::kColQsf + 4 * C::kQAtoms * t + 4 * kk, ksf + 4 * kk, kk > 0 ? 1u : 0u);
+                        else
+                            tc_mma_mxf4(t_s, qdesc + 2 * kk, kdesc + 2 * kk, mxf4_idesc(T, 2 * kk, 2 * kk),
+                                        tbase + C::kColQsf + 4 * t, ksf, kk > 0 ? 1u : 0u);
+                    }
                     tc_commit(bar_s_full + t);
                     if (t == NT - 1) tc_commit(bar_k_empty + s);
                 }
@@ -337,20 +374,35 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
             auto issue_pv = [&](int t, int j) -> bool {
                 const int s = j % S;
                 const uint32_t n = j / S;
+                const int slot = j % C::kSfSlots;
                 if (!wait(bar_p_full + t, j & 1)) return false;
                 if (t == 0 && !wait(bar_v_full + s, n & 1)) return false;
                 tc_fence_after_sync();
                 const uint64_t pdesc = pdesc0 + static_cast<uint32_t>(t * (C::kPBytes >> 4));
                 const uint64_t vdesc = vdesc0 + static_cast<uint32_t>(s * (C::kVStride >> 4));
+                const uint32_t psf_col = tbase + C::kColPsf + 4 * C::kVAtoms * t;
+                const uint32_t vsf_col = tbase + C::kColVsf + 8 * C::kVAtoms * slot;
                 if (leader) {
-                    tc_cp_sf(tbase + C::kColPsf + 4 * t, psf0 + static_cast<uint32_t>(t * (512 >> 4)));
-                    if (t == 0) tc_cp_sf(tbase + C::kColVsf + 8 * s, vsf0 + static_cast<uint32_t>(s * (512 >> 4)));
+#pragma unroll
+                    for (int a = 0; a < C::kVAtoms; ++a)
+                        tc_cp_sf(psf_col + 4 * a, psf0 + static_cast<uint32_t>((t * C::kPsfBytes + 512 * a) >> 4));
+                    if (t == 0) {
+#pragma unroll
+                        for (int a = 0; a < C::kVAtoms; ++a)
+                            tc_cp_sf(vsf_col + 8 * a, vsf0 + static_cast<uint32_t>((s * C::kVsfBytes + 512 * a) >> 4));
+                    }
 #pragma unroll
                     for (int kk = 0; kk < T / 64; ++kk) {
-                        const uint32_t sfb_id = (T == 64) ? 2u * (j & 1) : 2u * kk;
-                        tc_mma_mxf4(tbase + C::kColO + t * C::kOCols, pdesc + 2 * kk, vdesc + 2 * kk,
-                                    mxf4_idesc(D + 16, 2 * kk, sfb_id), tbase + C::kColPsf + 4 * t,
-                                    tbase + C::kColVsf + 8 * s, (j > 0 || kk > 0) ? 1u : 0u);
+                        if constexpr (NV) {
+                            tc_mma_nvf4(tbase + C::kColO + t * C::kOCols, pdesc + 2 * kk, vdesc + 2 * kk,
+                                        nvf4_idesc(D + 16), psf_col + 4 * kk, vsf_col + 8 * kk,
+                                        (j > 0 || kk > 0) ? 1u : 0u);
+                        } else {
+                            const uint32_t sfb_id = (T == 64) ? 2u * (j & 1) : 2u * kk;
+                            tc_mma_mxf4(tbase + C::kColO + t * C::kOCols, pdesc + 2 * kk, vdesc + 2 * kk,
+                                        mxf4_idesc(D + 16, 2 * kk, sfb_id), psf_col, vsf_col,
+                                        (j > 0 || kk > 0) ? 1u : 0u);
+                        }
                     }
                     tc_commit(bar_o_done + t);
                     if (t == NT - 1) tc_commit(bar_v_empty + s);
@@ -362,9 +414,14 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
             if (ok) {
                 tc_fence_after_sync();
                 if (leader) {
-                    for (int t = 0; t < NT; ++t) tc_cp_sf(tbase + C::kColQsf + 4 * t, sf_desc(sQsf + t * 512));
+                    for (int t = 0; t < NT; ++t)
+                        for (int a = 0; a < C::kQAtoms; ++a)
+                            tc_cp_sf(tbase + C::kColQsf + 4 * C::kQAtoms * t + 4 * a,
+                                     sf_desc(sQsf + t * C::kQsfBytes + 512 * a));
                     if (D == 128)
-                        for (int s = 0; s < S; ++s) tc_cp_sf(tbase + C::kColVsf + 8 * s + 4, sf_desc(sVsfConst));
+                        for (int slot = 0; slot < C::kSfSlots; ++slot)
+                            for (int a = 0; a < C::kVAtoms; ++a)
+                                tc_cp_sf(tbase + C::kColVsf + 8 * C::kVAtoms * slot + 8 * a + 4, sf_desc(sVsfConst));
                 }
                 __syncwarp();
             }
@@ -399,13 +456,21 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
         const int row = tid & 127;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t t_o = tbase + lane_base + C::kColO + t * C::kOCols;
-        const float kq = p.kq;
+        // NVFP4: S and O come out of the tensor core in units of the second-level
+        // scales 6 g (Q, K, V) and 6 * 448 (P); fold them into kq and the epilogue.
+        float kq = p.kq;
+        float o_unit = 1.f;
+        if constexpr (NV) {
+            const float Gq = __fmul_rn(6.f, p.gs[bh]), Gk = __fmul_rn(6.f, p.gs[p.BH + bh]);
+            kq = p.kq / (Gq * Gk);
+            o_unit = __fmul_rn(6.f, p.gs[2 * p.BH + bh]);
+        }
         const float e_sign = p.e_sign;
         const float e_off = p.e_off;
         const int e_add = p.e_add;
         const int valid_last = p.N - (nkv - 1) * T;
         uint8_t* sPt = sP + t * C::kPBytes;
-        uint8_t* sPsft = sPsf + t * 512;
+        uint8_t* sPsft = sPsf + t * C::kPsfBytes;
         float m_run = -INFINITY;
         float l_run = 0.f;  // PNQ off: the row sum of the unquantized exponentials
         bool ok = true;
@@ -431,58 +496,81 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                 for (int i = 0; i < T; ++i)
                     if (i >= valid_last) sv[i] = -INFINITY;
             }
-            float bm[T / 32];
+            constexpr int NBM = NV ? T / 16 : T / 32;  // blocks of P (16 or 32 keys)
+            float bm[NBM];
 #pragma unroll
-            for (int k = 0; k < T / 32; ++k) bm[k] = block_max32(sv + 32 * k);
+            for (int k = 0; k < NBM; ++k) bm[k] = NV ? block_max16(sv + 16 * k) : block_max32(sv + 32 * k);
             float tmax = bm[0];
 #pragma unroll
-            for (int k = 1; k < T / 32; ++k) tmax = fmaxf(tmax, bm[k]);
+            for (int k = 1; k < NBM; ++k) tmax = fmaxf(tmax, bm[k]);
             const float m_new = fmaxf(m_run, tmax);
             const bool rescale = (j > 0) && (m_new > m_run);
             const float alpha = rescale ? ex2_approx((m_run - m_new) * kq) : 1.f;
 
-            // PNQ: quantize exp(S - m_new) per 32-column block.  The block's largest
-            // exponential is 2^x with x = (bm - m_new) * kq; the scale rule is applied to
-            // it in the log domain (no exponential needed), and each element is then
-            // 2^(s*kq - (m*kq + e)), already divided by the block scale 2^e.
             uint32_t pw[T / 8];
-            uint32_t sfw = 0;
+            uint32_t sfw[C::kVAtoms];
+#pragma unroll
+            for (int a = 0; a < C::kVAtoms; ++a) sfw[a] = 0u;
             float lsum = 0.f;
+            // Per block of P: `nbias[k]` turns s * kq into the log2 of the element as it
+            // enters the E2M1 rounding, `back[k]` brings a rounded value back to exp(s - m_new).
+            float nbias[NBM], back[NBM];
+            if constexpr (NV) {
+                // NVFP4 P (blocks of 16 keys): scale sb = E4M3(pmax * 448) with pmax the block's
+                // largest exponential, element = exp(s - m_new) * 2688 / sb.  A block whose scale
+                // rounds to 0 holds values below 2.3e-6 and is left unscaled (all its codes are 0).
 #pragma unroll
-            for (int k = 0; k < T / 32; ++k) {
-                // x = (bm - m_new) * kq is exactly 0 for the block holding the row max, so
-                // the OCP boundary at integer x is decided exactly there.
-                float z = fmaf(e_sign, (bm[k] - m_new) * kq, e_off);
-                z = fminf(fmaxf(z, -250.f), 250.f);  // masked blocks give +-inf; any |z| > 127 clamps e below
-                const int fl = static_cast<int>(__float_as_uint(__fadd_rd(z, 12582912.f)) - 0x4B400000u);
-                int e = (e_sign > 0.f ? fl : -fl) + e_add;
-                e = e < -127 ? -127 : e;
-                const float nbias = -fmaf(m_new, kq, static_cast<float>(e));
-                float bsum = 0.f;
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    float f[8];
-#pragma unroll
-                    for (int i = 0; i < 8; i += 2) {
-                        float w0, w1;
-                        ffma2_bcast(w0, w1, sv[32 * k + 8 * g + i], sv[32 * k + 8 * g + i + 1], kq, nbias);
-                        if (!C::fma_pair(4 * g + i / 2, PNQ)) {  // MUFU
-                            f[i] = ex2_approx(w0);
-                            f[i + 1] = ex2_approx(w1);
-                        } else if constexpr (PNQ) {  // FMA pipe: only the E2M1 code is kept
-                            exp2_code_x2(w0, w1, f[i], f[i + 1]);
-                        } else {                     // FMA pipe: the value enters the row sum
-                            exp2_fma_x2(w0, w1, f[i], f[i + 1]);
-                        }
-                    }
-                    if constexpr (!PNQ) {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) bsum += f[i];
-                    }
-                    pw[4 * k + g] = pack_e2m1x8(f);
+                for (int k = 0; k < NBM; ++k) {
+                    const float pmax = ex2_approx((bm[k] - m_new) * kq);
+                    const uint32_t sb = e4m3_encode_sat(pmax * 448.f);
+                    const float sbv = e4m3_decode(sb);
+                    nbias[k] = fmaf(-m_new, kq, sbv > 0.f ? 11.392317422778761f - lg2_approx(sbv) : 0.f);
+                    back[k] = sbv > 0.f ? sbv * (1.f / 2688.f) : 1.f;
+                    sfw[k / 4] |= sb << (8 * (k % 4));
                 }
-                sfw |= static_cast<uint32_t>(e + 127) << (8 * k);
-                if constexpr (!PNQ) lsum = fmaf(bsum, exp2_neg_int(-e), lsum);
+            } else {
+                // MXFP4 P: the block's largest exponential is 2^x with x = (bm - m_new) * kq; the
+                // scale rule is applied to it in the log domain (no exponential needed), and each
+                // element is then 2^(s*kq - (m*kq + e)), already divided by the block scale 2^e.
+#pragma unroll
+                for (int k = 0; k < NBM; ++k) {
+                    // x = (bm - m_new) * kq is exactly 0 for the block holding the row max, so
+                    // the OCP boundary at integer x is decided exactly there.
+                    float z = fmaf(e_sign, (bm[k] - m_new) * kq, e_off);
+                    z = fminf(fmaxf(z, -250.f), 250.f);  // masked blocks give +-inf; any |z| > 127 clamps e below
+                    const int fl = static_cast<int>(__float_as_uint(__fadd_rd(z, 12582912.f)) - 0x4B400000u);
+                    int e = (e_sign > 0.f ? fl : -fl) + e_add;
+                    e = e < -127 ? -127 : e;
+                    nbias[k] = -fmaf(m_new, kq, static_cast<float>(e));
+                    back[k] = exp2_neg_int(-e);
+                    sfw[0] |= static_cast<uint32_t>(e + 127) << (8 * k);
+                }
+            }
+            // Elements, 8 at a time (group gg: keys 8 gg .. 8 gg + 7, P block gg / (NV ? 2 : 4)).
+#pragma unroll
+            for (int gg = 0; gg < T / 8; ++gg) {
+                const int k = NV ? gg / 2 : gg / 4;
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 8; i += 2) {
+                    float w0, w1;
+                    ffma2_bcast(w0, w1, sv[8 * gg + i], sv[8 * gg + i + 1], kq, nbias[k]);
+                    if (!C::fma_pair(4 * (gg % 4) + i / 2, PNQ)) {  // MUFU
+                        f[i] = ex2_approx(w0);
+                        f[i + 1] = ex2_approx(w1);
+                    } else if constexpr (PNQ) {  // FMA pipe: only the E2M1 code is kept
+                        exp2_code_x2(w0, w1, f[i], f[i + 1]);
+                    } else {                     // FMA pipe: the value enters the row sum
+                        exp2_fma_x2(w0, w1, f[i], f[i + 1]);
+                    }
+                }
+                if constexpr (!PNQ) {
+                    float gsum = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) gsum += f[i];
+                    lsum = fmaf(gsum, back[k], lsum);
+                }
+                pw[gg] = pack_e2m1x8(f);
             }
             // The P buffer and O are free once the previous P*V of this tile finished.
             if (j > 0) {
@@ -515,7 +603,9 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
                     *reinterpret_cast<uint4*>(prow + 16 * phys) =
                         make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
                 }
-                reinterpret_cast<uint32_t*>(sPsft)[(row & 31) * 4 + (row >> 5)] = sfw;
+#pragma unroll
+                for (int a = 0; a < C::kVAtoms; ++a)
+                    reinterpret_cast<uint32_t*>(sPsft + 512 * a)[(row & 31) * 4 + (row >> 5)] = sfw[a];
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
@@ -527,8 +617,9 @@ __global__ void __launch_bounds__(Cfg<D, T>::kThreads, 1)
         if (ok && __all_sync(0xffffffffu, mbar_wait_bounded(bar_o_done + t, (nkv - 1) & 1, abort_flag, p.status,
                                                              kTimeoutCode, kTimeoutNs))) {
             tc_fence_after_sync();
-            const float l = PNQ ? __uint_as_float(tmem_ld1_sync(t_o + D)) : l_run;
-            const float inv_l = 1.f / l;
+            // NVFP4: O and the PNQ row sum carry P's factor 2688 and O also V's 6 g.
+            const float l = PNQ ? __uint_as_float(tmem_ld1_sync(t_o + D)) : (NV ? 2688.f * l_run : l_run);
+            const float inv_l = 1.f / (l * o_unit);
             const int qrow = qp * C::kRows + t * 128 + row;
             float* out = p.O + (static_cast<size_t>(bh) * p.N + qrow) * D;
 #pragma unroll
@@ -577,18 +668,18 @@ bool encode_map(CUtensorMap* map, const void* base, uint64_t inner_bytes, uint64
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int T, bool PNQ>
+template <int D, int T, bool PNQ, bool NV>
 cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
-    using C = Cfg<D, T>;
+    using C = Cfg<D, T, NV>;
     static bool attr_set = false;
     if (!attr_set) {
         // The setmaxnreg split assumes the launch allocates exactly kLaunchRegs per
         // thread; with fewer, the softmax warpgroups' increase could never be met.
         cudaFuncAttributes fa{};
-        cudaError_t e = cudaFuncGetAttributes(&fa, mxattn_fwd_kernel<D, T, PNQ>);
+        cudaError_t e = cudaFuncGetAttributes(&fa, mxattn_fwd_kernel<D, T, PNQ, NV>);
         if (e != cudaSuccess) return e;
         if (fa.numRegs != static_cast<int>(C::kLaunchRegs)) return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, T, PNQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, T, PNQ, NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
@@ -613,8 +704,10 @@ cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
     kp.e_sign = a.qmax >= 8.f ? 1.f : -1.f;
     kp.e_off = a.qmax >= 8.f ? 0.f : static_cast<float>(std::log2(static_cast<double>(a.qmax)));
     kp.e_add = a.qmax >= 8.f ? -2 : 0;
+    kp.gs = a.gs;
+    kp.BH = static_cast<int>(a.BH);
     dim3 grid(static_cast<unsigned>(a.BH * kp.nq2));
-    mxattn_fwd_kernel<D, T, PNQ><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, kp);
+    mxattn_fwd_kernel<D, T, PNQ, NV><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, kp);
     return cudaGetLastError();
 }
 
@@ -622,7 +715,8 @@ cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
 
 template <int D, int T>
 cudaError_t launch_pnq(const AttnArgs& a, cudaStream_t stream) {
-    return a.pnq ? launch_impl<D, T, true>(a, stream) : launch_impl<D, T, false>(a, stream);
+    if (a.nv) return a.pnq ? launch_impl<D, T, true, true>(a, stream) : launch_impl<D, T, false, true>(a, stream);
+    return a.pnq ? launch_impl<D, T, true, false>(a, stream) : launch_impl<D, T, false, false>(a, stream);
 }
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {

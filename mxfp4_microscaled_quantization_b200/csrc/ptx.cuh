@@ -185,6 +185,20 @@ __device__ __forceinline__ void tc_mma_mxf4(uint32_t d_tmem, uint64_t a_desc, ui
         : "memory");
 }
 
+// The NVFP4 form: E2M1 operands with one E4M3 scale per 16 elements
+// (block16); the four scale bytes of a row for one K = 64 step sit in one
+// TMEM column, so the scale-factor ids are 0.
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
 #define MXATTN_R8(b) "=r"(v[b + 0]), "=r"(v[b + 1]), "=r"(v[b + 2]), "=r"(v[b + 3]), \
                      "=r"(v[b + 4]), "=r"(v[b + 5]), "=r"(v[b + 6]), "=r"(v[b + 7])
 #define MXATTN_W8(b) "r"(v[b + 0]), "r"(v[b + 1]), "r"(v[b + 2]), "r"(v[b + 3]), \
@@ -308,6 +322,21 @@ __host__ __device__ constexpr uint32_t mxf4_idesc(uint32_t n, uint32_t sfa_id, u
            | ((sfa_id & 3u) << 29);   // A scale-factor byte id
 }
 
+
+// Instruction descriptor of tcgen05.mma kind::mxf4nvf4 block16: M = 128, N = n,
+// E2M1 A and B, E4M3 scale factors (format bit 0), scale-factor ids 0.
+__host__ __device__ constexpr uint32_t nvf4_idesc(uint32_t n) {
+    return (1u << 7)                  // A format E2M1
+           | (1u << 10)               // B format E2M1
+           | ((n >> 3) << 17)         // N / 8
+           | ((128u >> 4) << 24);     // M / 16
+}
+
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // max(a, b, c) in one instruction (sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -438,6 +467,27 @@ __device__ __forceinline__ uint32_t pack_e2m1x8(const float (&x)[8]) {
         : "=r"(out)
         : "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]), "f"(x[4]), "f"(x[5]), "f"(x[6]), "f"(x[7]));
     return out;
+}
+
+// E4M3 (OCP FP8, no infinities) byte of a non-negative fp32 value: round to
+// nearest even, values at or above 448 saturate to 448 (0x7E).
+__device__ __forceinline__ uint32_t e4m3_encode_sat(float v) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(0.f), "f"(v));
+    return d & 0xFFu;
+}
+
+// E4M3 byte -> fp32 value (exact).
+__device__ __forceinline__ float e4m3_decode(uint32_t b) {
+    float f;
+    asm("{\n\t.reg .b16 lo, hi;\n\t.reg .b32 h2;\n\t"
+        "cvt.u16.u32 lo, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h2, lo;\n\t"
+        "mov.b32 {lo, hi}, h2;\n\t"
+        "cvt.f32.f16 %0, lo;\n\t}"
+        : "=f"(f)
+        : "r"(b));
+    return f;
 }
 
 // Block exponent from the bfloat16 bit pattern of a block maximum (>= 0)

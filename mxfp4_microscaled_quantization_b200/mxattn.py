@@ -71,6 +71,16 @@ def lib() -> ctypes.CDLL:
         L.mxattn_workspace_status.restype = i32
         L.mxattn_wait_selftest.argtypes = [i32, ctypes.c_uint, P, P]
         L.mxattn_wait_selftest.restype = i32
+        L.mxattn_nvfp4_quantize.argtypes = [P, i64, i64, P, P, P, P]
+        L.mxattn_nvfp4_quantize.restype = i32
+        L.mxattn_nvfp4_workspace_size.argtypes = [i32, i32, i32, i32]
+        L.mxattn_nvfp4_workspace_size.restype = u64
+        L.mxattn_nvfp4_forward.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f32, P, P, u64, P]
+        L.mxattn_nvfp4_forward.restype = i32
+        L.mxattn_nvfp4_prepare.argtypes = [P, P, P, i32, i32, i32, i32, P, u64, P]
+        L.mxattn_nvfp4_prepare.restype = i32
+        L.mxattn_nvfp4_attend.argtypes = [i32, i32, i32, i32, i32, i32, f32, P, P, u64, P]
+        L.mxattn_nvfp4_attend.restype = i32
         _lib = L
     return _lib
 
@@ -302,3 +312,86 @@ def attention_from_host(q_host, k_host, v_host, kv_tile=128, pnq=True, rule="uos
         out_host = torch.empty((B, H, N, d), dtype=torch.float32, pin_memory=True)
     out_host.copy_(od, non_blocking=True)
     return out_host
+
+
+# ---------------------------------------------------------------- NVFP4 comparison variant
+
+def mxattn_nvfp4_quantize(x: torch.Tensor, codes=None, scales=None, gs=None, stream=None):
+    """bf16 [..., cols] (cols % 16 == 0) -> (codes u8 [..., cols/2], E4M3 scales u8 [..., cols/16],
+    gs fp32 [2] = (amax, g)), one second-level scale g for the whole tensor."""
+    cols = x.shape[-1]
+    rows = x.numel() // cols if cols else 0
+    if codes is None:
+        codes = torch.empty(x.shape[:-1] + (cols // 2,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1] + (cols // 16,), dtype=torch.uint8, device=x.device)
+    if gs is None:
+        gs = torch.empty(2, dtype=torch.float32, device=x.device)
+    _check(lib().mxattn_nvfp4_quantize(_cuda(x, "x", torch.bfloat16), rows, cols, _cuda(codes, "codes"),
+                                       _cuda(scales, "scales"), _cuda(gs, "gs", torch.float32), _stream(stream)),
+           "mxattn_nvfp4_quantize")
+    return codes, scales, gs
+
+
+def nvfp4_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().mxattn_nvfp4_workspace_size(B, H, N, d))
+
+
+def nvfp4_workspace_layout(B: int, H: int, N: int, d: int) -> dict:
+    """Byte offsets of the NVFP4 workspace regions (as documented in include/mxattn.h)."""
+    a = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    BH, G, npad = B * H, (N + 127) // 128, (N + 31) // 32 * 32
+    off, out = 0, {}
+    for name, size in (("status", 256), ("q_codes", BH * N * d // 2), ("k_codes", BH * N * d // 2),
+                       ("vt_codes", BH * d * npad // 2), ("q_sf", BH * G * (d // 64) * 512),
+                       ("k_sf", BH * G * (d // 64) * 512), ("vt_sf", BH * G * 1024), ("amax", 3 * BH * 4),
+                       ("g", 3 * BH * 4)):
+        out[name] = (off, size)
+        off = a(off + size)
+    out["total"] = off
+    return out
+
+
+def new_nvfp4_workspace(B, H, N, d, device="cuda") -> torch.Tensor:
+    n = nvfp4_workspace_size(B, H, N, d)
+    if n == 0:
+        raise MxattnError(1, "mxattn_nvfp4_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def mxattn_nvfp4_forward(q, k, v, kv_tile=128, pnq=True, softmax_scale=0.0, out=None, workspace=None, stream=None):
+    """NVFP4 attention: q, k, v bf16 [B, H, N, d] -> O fp32 [B, H, N, d]."""
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_nvfp4_workspace(B, H, N, d, q.device)
+    _check(lib().mxattn_nvfp4_forward(_cuda(q, "q", torch.bfloat16), _cuda(k, "k", torch.bfloat16),
+                                      _cuda(v, "v", torch.bfloat16), B, H, N, d, kv_tile, 1 if pnq else 0,
+                                      float(softmax_scale), _cuda(out, "out", torch.float32),
+                                      _cuda(workspace, "workspace"), workspace.numel(), _stream(stream)),
+           "mxattn_nvfp4_forward")
+    return out
+
+
+def mxattn_nvfp4_prepare(q, k, v, workspace=None, stream=None):
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, H, N, d]")
+    if workspace is None:
+        workspace = new_nvfp4_workspace(B, H, N, d, q.device)
+    _check(lib().mxattn_nvfp4_prepare(_cuda(q, "q", torch.bfloat16), _cuda(k, "k", torch.bfloat16),
+                                      _cuda(v, "v", torch.bfloat16), B, H, N, d, _cuda(workspace, "workspace"),
+                                      workspace.numel(), _stream(stream)), "mxattn_nvfp4_prepare")
+    return workspace
+
+
+def mxattn_nvfp4_attend(workspace, B, H, N, d, kv_tile=128, pnq=True, softmax_scale=0.0, out=None, stream=None):
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.float32, device=workspace.device)
+    _check(lib().mxattn_nvfp4_attend(B, H, N, d, kv_tile, 1 if pnq else 0, float(softmax_scale),
+                                     _cuda(out, "out", torch.float32), _cuda(workspace, "workspace"),
+                                     workspace.numel(), _stream(stream)), "mxattn_nvfp4_attend")
+    return out

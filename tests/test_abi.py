@@ -99,3 +99,36 @@ def test_qmax_entry_points_reject_boundaries_outside_the_family(L):
         assert L.mxattn_prepare_qmax(fake, fake, fake, 1, 1, 256, 64, f(q), fake, ws_ok, None) == 1
         assert L.mxattn_attend_qmax(1, 1, 256, 64, 64, 1, f(q), f(0.0), fake, fake, ws_ok, None) == 1
     assert L.mxattn_quantize_qmax(None, 0, 64, f(6.0), None, None, None) == 0  # empty, valid boundary
+
+
+def test_nvfp4_workspace_size_matches_documented_layout(L):
+    for shape in ((1, 1, 256, 64), (1, 8, 4096, 128), (1, 40, 32760, 128), (2, 3, 1, 64), (1, 1, 129, 128)):
+        assert mx.nvfp4_workspace_size(*shape) == mx.nvfp4_workspace_layout(*shape)["total"]
+    assert mx.nvfp4_workspace_size(1, 1, 256, 96) == 0
+    assert mx.nvfp4_workspace_size(1, 1, 0, 64) == 0
+
+
+def test_nvfp4_entry_points_reject_bad_arguments_before_launching(L):
+    fake = _p(1 << 20)
+    f = ctypes.c_float
+    assert L.mxattn_nvfp4_quantize(fake, 4, 40, fake, fake, fake, None) == 1   # cols % 16 != 0
+    assert L.mxattn_nvfp4_quantize(fake, -1, 64, fake, fake, fake, None) == 1  # negative rows
+    assert L.mxattn_nvfp4_quantize(None, 4, 64, fake, fake, fake, None) == 1   # null input
+    assert L.mxattn_nvfp4_quantize(fake, 4, 64, fake, fake, None, None) == 1   # null gs
+    assert L.mxattn_nvfp4_quantize(_p((1 << 20) + 8), 4, 64, fake, fake, fake, None) == 1  # misaligned
+    assert L.mxattn_nvfp4_quantize(None, 0, 64, None, None, None, None) == 0   # empty is a no-op
+    ws_ok = mx.nvfp4_workspace_size(1, 1, 256, 64)
+    args = lambda d=64, t=64, pnq=1, N=256, ws=ws_ok, o=fake, H=1: (  # noqa: E731
+        fake, fake, fake, 1, H, N, d, t, pnq, f(0.0), o, fake, ws, None)
+    assert L.mxattn_nvfp4_forward(*args(d=96)) == 2
+    assert L.mxattn_nvfp4_forward(*args(t=32)) == 2
+    assert L.mxattn_nvfp4_forward(*args(pnq=2)) == 1
+    assert L.mxattn_nvfp4_forward(*args(N=0)) == 1
+    assert L.mxattn_nvfp4_forward(*args(ws=ws_ok - 1)) == 1
+    assert L.mxattn_nvfp4_forward(*args(o=None)) == 1
+    assert L.mxattn_nvfp4_forward(*args(H=65536, ws=1 << 40)) == 2
+    # an MXFP4-sized workspace is too small for the NVFP4 layout of the same shape
+    assert mx.mxattn_workspace_size(1, 1, 256, 128) < mx.nvfp4_workspace_size(1, 1, 256, 128)
+    assert L.mxattn_nvfp4_prepare(fake, fake, fake, 1, 1, 256, 128, fake, mx.mxattn_workspace_size(1, 1, 256, 128),
+                                  None) == 1
+    assert L.mxattn_nvfp4_attend(1, 1, 256, 64, 64, 1, f(0.0), fake, fake, ws_ok - 1, None) == 1
