@@ -316,7 +316,15 @@ def qmax_study(args):
                 got = o[:, :, rows].double()
                 rel = float((got - exact).norm() / exact.norm())
                 out_rows.append({"inputs": name, "qmax": qmax, "pnq": pnq, "rel_err": rel})
-    line = {"study": "scale boundary Qmax vs O error against exact fp64 attention",
+        wsn = mx.new_nvfp4_workspace(B, H, N, d)
+        for pnq in (True, False):
+            o = mx.mxattn_nvfp4_forward(q, k, v, 128, pnq, workspace=wsn)
+            torch.cuda.synchronize()
+            if mx.mxattn_workspace_status(wsn) != 0:
+                raise RuntimeError("NVFP4 attention kernel reported a timeout")
+            rel = float((o[:, :, rows].double() - exact).norm() / exact.norm())
+            out_rows.append({"inputs": name, "qmax": "nvfp4", "pnq": pnq, "rel_err": rel})
+    line = {"study": "scale boundary Qmax (and the NVFP4 variant) vs O error against exact fp64 attention",
             "shapes": "gaussian / student_t3 / outlier: B=1 H=8 N=4096 d=128; video_dit_4heads: B=1 H=4 "
                       "N=32760 d=128; kv_tile 128; 512 seeded query rows per head",
             "rows": out_rows}
@@ -360,16 +368,23 @@ def run_gpu(args, rank, world, local_rank):
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)  # noqa: E731
     q, k, v = to_dev(Q), to_dev(K), to_dev(V)
     out = torch.empty((B, H, N, d), dtype=torch.float32, device="cuda")
-    ws = mx.new_workspace(B, H, N, d)
+    nv_step = args.format == "nvfp4"
+    ws = mx.new_nvfp4_workspace(B, H, N, d) if nv_step else mx.new_workspace(B, H, N, d)
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        mx.mxattn_prepare(q, k, v, "uos", ws)
+        if nv_step:
+            mx.mxattn_nvfp4_prepare(q, k, v, ws)
+        else:
+            mx.mxattn_prepare(q, k, v, "uos", ws)
         if ev is not None:
             ev[1].record(stream)
-        mx.mxattn_attend(ws, B, H, N, d, w.kv_tile, True, "uos", 0.0, out)
+        if nv_step:
+            mx.mxattn_nvfp4_attend(ws, B, H, N, d, w.kv_tile, True, 0.0, out)
+        else:
+            mx.mxattn_attend(ws, B, H, N, d, w.kv_tile, True, "uos", 0.0, out)
         if ev is not None:
             ev[2].record(stream)
 
@@ -424,6 +439,31 @@ def run_gpu(args, rank, world, local_rank):
         overhead = {"ocp_no_pnq_attn_ms": ocp_ms, "uos_pnq_attn_ms": attn_avg_ms,
                     "uos_pnq_over_ocp": attn_avg_ms / ocp_ms - 1.0}
 
+    # The NVFP4 comparison variant (16-element blocks, E4M3 scales, per-head fp32
+    # scales) on the same workload and kernel structure, PNQ on.
+    nvfp4 = None
+    if not args.quick:
+        wsn = mx.new_nvfp4_workspace(B, H, N, d)
+        mx.mxattn_nvfp4_prepare(q, k, v, wsn)
+        mx.mxattn_nvfp4_attend(wsn, B, H, N, d, w.kv_tile, True, 0.0, out)
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(5)]
+        for e in ev:
+            e[0].record(stream)
+            mx.mxattn_nvfp4_prepare(q, k, v, wsn)
+            e[1].record(stream)
+            mx.mxattn_nvfp4_attend(wsn, B, H, N, d, w.kv_tile, True, 0.0, out)
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        if mx.mxattn_workspace_status(wsn) != 0:
+            raise RuntimeError("NVFP4 attention kernel reported a timeout")
+        nv_prep, nv_attn = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in ev) / len(ev),
+                                           sum(e[1].elapsed_time(e[2]) for e in ev) / len(ev)], dist, "cuda")
+        nvfp4 = {"prepare_ms": nv_prep, "attn_ms": nv_attn, "attn_tflops": w.flops / (nv_attn / 1e3) / 1e12,
+                 "step_tflops": w.flops / ((nv_prep + nv_attn) / 1e3) / 1e12,
+                 "uos_pnq_attn_speedup": nv_attn / attn_avg_ms, "kernel": f"mxattn_fwd_kernel<{w.d},{w.kv_tile},1,nvfp4>"}
+        del wsn
+
     if rank == 0:
         attn_tflops = w.flops / (attn_avg_ms / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
@@ -432,14 +472,16 @@ def run_gpu(args, rank, world, local_rank):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "strong" if args.shard == "heads" else "weak",
-            "vs_baseline": None, "dtype": "mxfp4 (e2m1 x e8m0, fp32 accumulate)", "data": "synthetic",
+            "vs_baseline": None, "data": "synthetic",
+            "dtype": ("nvfp4 (e2m1 x e4m3, fp32 accumulate)" if nv_step else "mxfp4 (e2m1 x e8m0, fp32 accumulate)"),
             "config": {**config_dict(w_full), "parallelism": (
                 f"heads sharded over {world} ranks (one problem, no exchange)" if args.shard == "heads"
                 else f"{world} independent replicas (one batch per rank)")},
             "pct_of_fp4_peak": 100.0 * value / world / peak,
-            "roofline": {"bound": "tensor", "kernel": f"mxattn_fwd_kernel<{w.d},{w.kv_tile}>", "achieved": attn_tflops,
+            "roofline": {"bound": "tensor", "achieved": attn_tflops,
+                         "kernel": f"mxattn_fwd_kernel<{w.d},{w.kv_tile}{',nvfp4' if nv_step else ''}>",
                          "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
-                         "traffic": profiled_traffic() if w == WORKLOAD else None,
+                         "traffic": profiled_traffic() if (w == WORKLOAD and not nv_step) else None,
                          "peak_source": f"{peak_kind} bf16 sustained {peaks['bf16_tflops_sustained']} TFLOP/s x "
                                         f"{FP4_PER_BF16:g} (nominal dense fp4:bf16)",
                          "attn_ms": attn_avg_ms, "prepare_ms": sum(prep_ms) / len(prep_ms),
@@ -451,7 +493,8 @@ def run_gpu(args, rank, world, local_rank):
                 "ms_per_step": e2e_ms, "api": "attention_from_host -> mxattn_forward"},
             "mufu_roofline": mufu_roofline(w, attn_avg_ms, clocks),
             "uos_pnq_overhead": overhead,
-            "gpu_launches": 3 * args.steps,
+            "nvfp4": nvfp4,
+            "gpu_launches": (4 if nv_step else 3) * args.steps,
             "clocks": clocks,
             "quantize_sweep": quant,
         }
@@ -499,6 +542,8 @@ def main():
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N > 1: one independent batch per rank (weak scaling, default) or the heads of one "
                          "problem split over the ranks (strong scaling)")
+    ap.add_argument("--format", choices=["mxfp4", "nvfp4"], default="mxfp4",
+                    help="operand format of the timed step (nvfp4: the comparison variant; only with --quick)")
     ap.add_argument("--qmax-study", action="store_true",
                     help="instead of the timed step: O error against exact attention over scale boundaries in [6, 8]")
     ap.add_argument("--quick", action="store_true",
@@ -508,6 +553,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     args.warmup = max(args.warmup, 3)  # timing rule: at least 3 warm-up steps
+    if args.format == "nvfp4" and not args.quick:
+        ap.error("--format nvfp4 times the comparison variant alone and needs --quick")
     if args.impl == "reference":
         return run_reference(args, rank, world)
     if args.qmax_study:
