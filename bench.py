@@ -490,7 +490,8 @@ def run_gpu(args, rank, world, local_rank):
             "e2e": None if e2e_ms is None else {
                 "value": job_flops / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": 3 * B * H * N * d * 2, "d2h_bytes_per_step": B * H * N * d * 4,
-                "ms_per_step": e2e_ms, "api": "attention_from_host -> mxattn_forward"},
+                "ms_per_step": e2e_ms, "api": "attention_from_host -> mxattn_forward",
+                "pipeline": "16 groups of (batch, head) slices; H2D, attention and D2H overlap on three streams"},
             "mufu_roofline": mufu_roofline(w, attn_avg_ms, clocks),
             "uos_pnq_overhead": overhead,
             "nvfp4": nvfp4,

@@ -292,25 +292,73 @@ def mxattn_status_string(status: int) -> str:
     return status_string(status)
 
 
+_side_streams = {}
+
+
+def _copy_streams(device):
+    """Two side streams per device for the host<->device copies of attention_from_host."""
+    key = torch.device(device).index
+    if key not in _side_streams:
+        _side_streams[key] = (torch.cuda.Stream(device), torch.cuda.Stream(device))
+    return _side_streams[key]
+
+
 def attention_from_host(q_host, k_host, v_host, kv_tile=128, pnq=True, rule="uos", softmax_scale=0.0,
-                        device_buffers=None, out_host=None, stream=None):
-    """End-to-end call with host tensors: copy q, k, v (pinned host bf16) to the
-    device, run mxattn_forward, copy O back into `out_host` (pinned fp32).
-    `device_buffers` = (q, k, v, out, workspace) device tensors to reuse."""
+                        device_buffers=None, out_host=None, stream=None, chunks=16):
+    """End-to-end call with host tensors: q, k, v (pinned host bf16 [B, H, N, d])
+    to the device, mxattn_forward, O back into `out_host` (pinned fp32).
+
+    The (batch, head) slices are processed in `chunks` groups, pipelined over
+    three streams: the copy of group i+1 to the device and of group i-1 back to
+    the host overlap the attention of group i (heads are independent, so each
+    group is one mxattn_forward call on a contiguous slice).  The work is
+    ordered on `stream` (default: the current stream): everything, including
+    the last copy back, is done when `stream` reaches the point after this call.
+    `device_buffers` = (q, k, v, out, workspace) device tensors to reuse; the
+    workspace needs only the size of one group."""
     B, H, N, d = q_host.shape
+    BH = B * H
+    dev = torch.device("cuda", torch.cuda.current_device())
     if device_buffers is None:
-        dev = torch.device("cuda")
-        device_buffers = (torch.empty_like(q_host, device=dev), torch.empty_like(k_host, device=dev),
-                          torch.empty_like(v_host, device=dev),
-                          torch.empty((B, H, N, d), dtype=torch.float32, device=dev), new_workspace(B, H, N, d))
+        device_buffers = (torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                          torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                          torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                          torch.empty((B, H, N, d), dtype=torch.float32, device=dev), None)
     qd, kd, vd, od, ws = device_buffers
-    qd.copy_(q_host, non_blocking=True)
-    kd.copy_(k_host, non_blocking=True)
-    vd.copy_(v_host, non_blocking=True)
-    mxattn_forward(qd, kd, vd, kv_tile, pnq, rule, softmax_scale, od, ws, stream)
     if out_host is None:
         out_host = torch.empty((B, H, N, d), dtype=torch.float32, pin_memory=True)
-    out_host.copy_(od, non_blocking=True)
+    n_chunks = max(1, min(int(chunks), BH))
+    per = -(-BH // n_chunks)
+    if ws is None:
+        ws = new_workspace(1, per, N, d, dev)
+    compute = torch.cuda.current_stream(dev) if stream is None else stream
+    h2d, d2h = _copy_streams(dev)
+    h2d.wait_stream(compute)  # the device buffers may still be in use by earlier work on `stream`
+    d2h.wait_stream(compute)
+    flat = lambda t: t.view(BH, N, d)  # noqa: E731
+    qh, kh, vh, oh = flat(q_host), flat(k_host), flat(v_host), flat(out_host)
+    qf, kf, vf, of = flat(qd), flat(kd), flat(vd), flat(od)
+    last = None
+    for c0 in range(0, BH, per):
+        sl = slice(c0, min(BH, c0 + per))
+        with torch.cuda.stream(h2d):
+            qf[sl].copy_(qh[sl], non_blocking=True)
+            kf[sl].copy_(kh[sl], non_blocking=True)
+            vf[sl].copy_(vh[sl], non_blocking=True)
+            loaded = torch.cuda.Event()
+            loaded.record(h2d)
+        compute.wait_event(loaded)
+        nh = sl.stop - sl.start
+        mxattn_forward(qf[sl].view(1, nh, N, d), kf[sl].view(1, nh, N, d), vf[sl].view(1, nh, N, d), kv_tile, pnq,
+                       rule, softmax_scale, of[sl].view(1, nh, N, d), ws, compute)
+        done = torch.cuda.Event()
+        done.record(compute)
+        d2h.wait_event(done)
+        with torch.cuda.stream(d2h):
+            oh[sl].copy_(of[sl], non_blocking=True)
+            last = torch.cuda.Event()
+            last.record(d2h)
+    compute.wait_event(last)
     return out_host
 
 

@@ -237,3 +237,15 @@ def test_status_string_roundtrip():
     assert mx.mxattn_status_string(0) == "ok"
     assert "timed out" in mx.mxattn_status_string(4)
     assert math.isfinite(mx.mxattn_workspace_size(1, 40, 32760, 128))
+
+
+@pytest.mark.parametrize("chunks", [1, 3, 8, 100])
+def test_attention_from_host_pipeline_matches_forward(chunks):
+    """The host-to-host call (head groups pipelined over three streams) gives the
+    same O as one mxattn_forward on device tensors, bit for bit."""
+    Q, K, V = wl.gaussian_qkv(2, 5, 300, 128, seed=31)
+    ref, _ = run_forward(Q, K, V, 128, True, "uos")
+    host = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()  # noqa: E731
+    out = mx.attention_from_host(host(Q), host(K), host(V), 128, True, "uos", chunks=chunks)
+    torch.cuda.current_stream().synchronize()
+    np.testing.assert_array_equal(out.numpy().astype(np.float64), ref)
