@@ -356,14 +356,25 @@ def run_gpu(args, rank, world, local_rank):
             raise ValueError(f"{w_full.H} heads cannot be sharded over {world} ranks")
         Q, K, V = (np.ascontiguousarray(a[:, lo:hi]) for a in wl.make_qkv(w_full, seed=0))
         w = dataclasses.replace(w_full, H=hi - lo)
+    elif args.shard == "sequence":
+        # One problem, its tokens split over the ranks (sequence parallelism): an
+        # all-to-all regroups Q, K, V by head before the attention and O by token after.
+        import dataclasses
+
+        if w_full.H % world or w_full.N % world:
+            raise ValueError(f"H={w_full.H} and N={w_full.N} must divide by the {world} ranks")
+        n = w_full.N // world
+        Q, K, V = (np.ascontiguousarray(a[:, :, rank * n:(rank + 1) * n]) for a in wl.make_qkv(w_full, seed=0))
+        w = dataclasses.replace(w_full, H=w_full.H // world)  # what the kernels see after the exchange
     else:
         w = w_full
         Q, K, V = wl.make_qkv(w, seed=rank_seed(rank))
+    seq = args.shard == "sequence"
     B, H, N, d = w.B, w.H, w.N, w.d
     # whole-job work per step: every rank's problem (replicas) or the one sharded problem
-    job_flops = w_full.flops if args.shard == "heads" else world * w.flops
+    job_flops = w_full.flops if args.shard in ("heads", "sequence") else world * w.flops
     base = None
-    if rank == 0 and not args.quick:
+    if rank == 0 and not args.quick and not seq:
         base = cpu_baseline(Q, K, V, w, budget_s=args.cpu_budget)
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)  # noqa: E731
     q, k, v = to_dev(Q), to_dev(K), to_dev(V)
@@ -372,13 +383,17 @@ def run_gpu(args, rank, world, local_rank):
     ws = mx.new_nvfp4_workspace(B, H, N, d) if nv_step else mx.new_workspace(B, H, N, d)
     stream = torch.cuda.current_stream()
 
+    if seq:
+        from mxfp4_microscaled_quantization_b200 import ulysses
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
+        qs, ks, vs = (ulysses.seq_to_head(t) for t in (q, k, v)) if seq else (q, k, v)
         if nv_step:
-            mx.mxattn_nvfp4_prepare(q, k, v, ws)
+            mx.mxattn_nvfp4_prepare(qs, ks, vs, ws)
         else:
-            mx.mxattn_prepare(q, k, v, "uos", ws)
+            mx.mxattn_prepare(qs, ks, vs, "uos", ws)
         if ev is not None:
             ev[1].record(stream)
         if nv_step:
@@ -387,6 +402,10 @@ def run_gpu(args, rank, world, local_rank):
             mx.mxattn_attend(ws, B, H, N, d, w.kv_tile, True, "uos", 0.0, out)
         if ev is not None:
             ev[2].record(stream)
+        if seq:
+            ulysses.head_to_seq(out)  # this rank's tokens of O
+        if ev is not None:
+            ev[3].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -394,7 +413,7 @@ def run_gpu(args, rank, world, local_rank):
     if mx.mxattn_workspace_status(ws) != 0:
         raise RuntimeError("attention kernel reported a timeout during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -404,7 +423,7 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    total_ms = evs[0][0].elapsed_time(evs[-1][2])
+    total_ms = evs[0][0].elapsed_time(evs[-1][3])
     attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
     prep_ms = [e[0].elapsed_time(e[1]) for e in evs]
     if mx.mxattn_workspace_status(ws) != 0:
@@ -414,17 +433,17 @@ def run_gpu(args, rank, world, local_rank):
     value = job_flops / (ms_per_step / 1e3) / 1e12
 
     e2e_ms = None
-    if not args.quick:
+    if not args.quick and not seq:
         e2e_ms = measure_e2e(torch, mx, Q, K, V, w, (q, k, v, out, ws), stream, args, dist)
 
     quant = None
-    if rank == 0 and not args.quick and not args.no_quantize_sweep:
+    if rank == 0 and not args.quick and not args.no_quantize_sweep and not seq:
         quant = quantize_sweep_point(torch, mx, peaks, peak_kind)
 
     # The same attention step with the OCP rule and no PNQ (the comparator the
     # method is measured against): the cost of UOS + PNQ relative to it.
     overhead = None
-    if not args.quick:
+    if not args.quick and not seq:
         mx.mxattn_prepare(q, k, v, "ocp", ws)
         for _ in range(2):
             mx.mxattn_attend(ws, B, H, N, d, w.kv_tile, False, "ocp", 0.0, out)
@@ -442,7 +461,7 @@ def run_gpu(args, rank, world, local_rank):
     # The NVFP4 comparison variant (16-element blocks, E4M3 scales, per-head fp32
     # scales) on the same workload and kernel structure, PNQ on.
     nvfp4 = None
-    if not args.quick:
+    if not args.quick and not seq:
         wsn = mx.new_nvfp4_workspace(B, H, N, d)
         mx.mxattn_nvfp4_prepare(q, k, v, wsn)
         mx.mxattn_nvfp4_attend(wsn, B, H, N, d, w.kv_tile, True, 0.0, out)
@@ -471,12 +490,13 @@ def run_gpu(args, rank, world, local_rank):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "strong" if args.shard == "heads" else "weak",
+            "scaling": "strong" if args.shard in ("heads", "sequence") else "weak",
             "vs_baseline": None, "data": "synthetic",
             "dtype": ("nvfp4 (e2m1 x e4m3, fp32 accumulate)" if nv_step else "mxfp4 (e2m1 x e8m0, fp32 accumulate)"),
-            "config": {**config_dict(w_full), "parallelism": (
-                f"heads sharded over {world} ranks (one problem, no exchange)" if args.shard == "heads"
-                else f"{world} independent replicas (one batch per rank)")},
+            "config": {**config_dict(w_full), "parallelism": {
+                "heads": f"heads sharded over {world} ranks (one problem, no exchange)",
+                "sequence": f"tokens sharded over {world} ranks (one problem; all-to-all to heads and back, NCCL)",
+                "replicas": f"{world} independent replicas (one batch per rank)"}[args.shard]},
             "pct_of_fp4_peak": 100.0 * value / world / peak,
             "roofline": {"bound": "tensor", "achieved": attn_tflops,
                          "kernel": f"mxattn_fwd_kernel<{w.d},{w.kv_tile}{',nvfp4' if nv_step else ''}>",
@@ -540,9 +560,10 @@ def main():
     ap.add_argument("--workload", choices=sorted(wl.WORKLOADS), default="video_dit",
                     help="workload to time (default: the video-DiT configuration the metric is quoted on)")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller cases for profiling)")
-    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
-                    help="N > 1: one independent batch per rank (weak scaling, default) or the heads of one "
-                         "problem split over the ranks (strong scaling)")
+    ap.add_argument("--shard", choices=["replicas", "heads", "sequence"], default="replicas",
+                    help="N > 1: one independent batch per rank (weak scaling, default); the heads of one problem "
+                         "split over the ranks; or its tokens split over the ranks with an all-to-all before and "
+                         "after the attention (strong scaling)")
     ap.add_argument("--format", choices=["mxfp4", "nvfp4"], default="mxfp4",
                     help="operand format of the timed step (nvfp4: the comparison variant; only with --quick)")
     ap.add_argument("--qmax-study", action="store_true",

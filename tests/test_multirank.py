@@ -81,3 +81,51 @@ def test_head_range_partitions_the_heads(H, world):
     assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
     sizes = [hi - lo for lo, hi in ranges]
     assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 0
+
+
+def _ulysses_worker(rank, world, port, out_dir):
+    import torch
+
+    import oracle
+    from mxfp4_microscaled_quantization_b200 import ulysses
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        Q, K, V = wl.gaussian_qkv(1, 4, 192, 64, seed=3)
+        n = 192 // world
+        local = lambda a: torch.from_numpy(np.ascontiguousarray(a[:, :, rank * n:(rank + 1) * n]).view(np.int16))  # noqa: E731
+
+        def oracle_attend(q, k, v, kv_tile):  # the CPU oracle stands in for the GPU kernel
+            bits = lambda t: np.ascontiguousarray(t.numpy()).view(np.uint16)  # noqa: E731
+            return torch.from_numpy(oracle.attention(bits(q), bits(k), bits(v), kv_tile, rule="uos", pnq=True))
+
+        o = ulysses.sequence_parallel_attention(local(Q), local(K), local(V), attend=oracle_attend, kv_tile=64)
+        np.save(os.path.join(out_dir, f"o{rank}.npy"), o.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_gloo_sequence_parallel_attention_equals_single_rank(world, tmp_path):
+    """Ulysses: tokens split over the ranks, all-to-all to heads, attention (the
+    oracle here, on CPU), all-to-all back; the ranks' token blocks put together
+    equal the single-rank result, bit for bit (same heads, same key-tile order)."""
+    import oracle
+
+    mp.start_processes(_ulysses_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       start_method="spawn")
+    Q, K, V = wl.gaussian_qkv(1, 4, 192, 64, seed=3)
+    ref = oracle.attention(Q, K, V, 64, rule="uos", pnq=True)
+    got = np.concatenate([np.load(tmp_path / f"o{r}.npy") for r in range(world)], axis=2)
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_sequence_layout_transforms_are_identity_on_one_rank():
+    import torch
+
+    from mxfp4_microscaled_quantization_b200 import ulysses
+
+    x = torch.arange(2 * 4 * 6 * 8, dtype=torch.float32).reshape(2, 4, 6, 8)
+    assert ulysses.seq_to_head(x) is x and ulysses.head_to_seq(x) is x
