@@ -50,6 +50,12 @@ namespace {
 
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
 constexpr uint32_t kTimeoutCode = 4u;           // MXATTN_ERR_TIMEOUT
+#ifndef MXATTN_NV_FMA_PNQ
+#define MXATTN_NV_FMA_PNQ 7
+#endif
+#ifndef MXATTN_NV_FMA_NOPNQ
+#define MXATTN_NV_FMA_NOPNQ 6
+#endif
 #ifndef MXATTN_ROLE_WAIT_HINT_NS
 #define MXATTN_ROLE_WAIT_HINT_NS 0
 #endif
@@ -99,7 +105,7 @@ struct Cfg {
     // exp2_code_x2), 6 without (the full polynomial, exp2_fma_x2); pair q is
     // one of them when (q * n) mod 16 < n, which spreads them evenly.
     __host__ __device__ static constexpr bool fma_pair(int q, bool pnq) {
-        const int n = pnq ? 7 : 6;
+        const int n = NV ? (pnq ? MXATTN_NV_FMA_PNQ : MXATTN_NV_FMA_NOPNQ) : (pnq ? 7 : 6);
         return (q * n) % 16 < n;
     }
 
@@ -524,7 +530,13 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
                     const float pmax = ex2_approx((bm[k] - m_new) * kq);
                     const uint32_t sb = e4m3_encode_sat(pmax * 448.f);
                     const float sbv = e4m3_decode(sb);
-                    nbias[k] = fmaf(-m_new, kq, sbv > 0.f ? 11.392317422778761f - lg2_approx(sbv) : 0.f);
+                    // log2(sbv) = exponent + log2(significand): lg2.approx only sees [1, 2), where its
+                    // absolute error is smallest, so the scaled elements keep fp32 accuracy at the
+                    // E2M1 rounding points (sbv is a normal fp32 number whenever it is not 0).
+                    const uint32_t sbits = __float_as_uint(sbv);
+                    const float l2 = static_cast<float>(static_cast<int>(sbits >> 23) - 127) +
+                                     lg2_approx(__uint_as_float((sbits & 0x7FFFFFu) | 0x3F800000u));
+                    nbias[k] = fmaf(-m_new, kq, sbv > 0.f ? 11.392317422778761f - l2 : 0.f);  // log2(2688) - log2(sbv)
                     back[k] = sbv > 0.f ? sbv * (1.f / 2688.f) : 1.f;
                     sfw[k / 4] |= sb << (8 * (k % 4));
                 }
