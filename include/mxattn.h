@@ -300,6 +300,24 @@ mxattn_status mxattn_nvfp4_prepare(const void* Q, const void* K, const void* V, 
 mxattn_status mxattn_nvfp4_attend(int B, int H, int N, int d, int kv_tile, int pnq, float softmax_scale, float* O,
                                   void* workspace, size_t workspace_bytes, mxattn_stream_t stream);
 
+/*
+ * Self-test of the softmax's decisions on P (this library's own check; the
+ * paper has no counterpart).  Runs, on n inputs, the device functions the
+ * attention kernel uses for P, so they can be compared with a reference:
+ *   path 0, 1, 2: in = w (fp32), out = E2M1 code (0..15) of 2^w computed by
+ *     ex2.approx (0), by the FMA-pipe code-only stand-in used with PNQ (1),
+ *     or by the FMA-pipe degree-5 exponential used without PNQ (2), each
+ *     rounded by cvt.rn.satfinite.e2m1x2;
+ *   path 3: in = x (log2 of a block's largest exponential, <= 0), out = the
+ *     MXFP4 block exponent e for the scale boundary qmax in (4, 8] (8 = OCP);
+ *   path 4: in = x, out = the NVFP4 block scale byte E4M3(2^x * 448).
+ *   in: device fp32 [n], out: device i32 [n], both 4-byte aligned; n % 8 == 0.
+ * Errors: MXATTN_ERR_INVALID (path, n, qmax for path 3, null or misaligned
+ * pointers), MXATTN_ERR_CUDA (launch failed).  Asynchronous on `stream`.
+ */
+mxattn_status mxattn_p_selftest(int path, const float* in, int64_t n, float qmax, int32_t* out,
+                                mxattn_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* mxattn_status_string(mxattn_status status);
 

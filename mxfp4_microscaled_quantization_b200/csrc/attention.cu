@@ -527,16 +527,9 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
                 // rounds to 0 holds values below 2.3e-6 and is left unscaled (all its codes are 0).
 #pragma unroll
                 for (int k = 0; k < NBM; ++k) {
-                    const float pmax = ex2_approx((bm[k] - m_new) * kq);
-                    const uint32_t sb = e4m3_encode_sat(pmax * 448.f);
-                    const float sbv = e4m3_decode(sb);
-                    // log2(sbv) = exponent + log2(significand): lg2.approx only sees [1, 2), where its
-                    // absolute error is smallest, so the scaled elements keep fp32 accuracy at the
-                    // E2M1 rounding points (sbv is a normal fp32 number whenever it is not 0).
-                    const uint32_t sbits = __float_as_uint(sbv);
-                    const float l2 = static_cast<float>(static_cast<int>(sbits >> 23) - 127) +
-                                     lg2_approx(__uint_as_float((sbits & 0x7FFFFFu) | 0x3F800000u));
-                    nbias[k] = fmaf(-m_new, kq, sbv > 0.f ? 11.392317422778761f - l2 : 0.f);  // log2(2688) - log2(sbv)
+                    float sbv, lf;
+                    const uint32_t sb = nv_p_block_scale((bm[k] - m_new) * kq, sbv, lf);
+                    nbias[k] = fmaf(-m_new, kq, lf);
                     back[k] = sbv > 0.f ? sbv * (1.f / 2688.f) : 1.f;
                     sfw[k / 4] |= sb << (8 * (k % 4));
                 }
@@ -548,11 +541,7 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
                 for (int k = 0; k < NBM; ++k) {
                     // x = (bm - m_new) * kq is exactly 0 for the block holding the row max, so
                     // the OCP boundary at integer x is decided exactly there.
-                    float z = fmaf(e_sign, (bm[k] - m_new) * kq, e_off);
-                    z = fminf(fmaxf(z, -250.f), 250.f);  // masked blocks give +-inf; any |z| > 127 clamps e below
-                    const int fl = static_cast<int>(__float_as_uint(__fadd_rd(z, 12582912.f)) - 0x4B400000u);
-                    int e = (e_sign > 0.f ? fl : -fl) + e_add;
-                    e = e < -127 ? -127 : e;
+                    const int e = p_block_exponent((bm[k] - m_new) * kq, e_sign, e_off, e_add);
                     nbias[k] = -fmaf(m_new, kq, static_cast<float>(e));
                     back[k] = exp2_neg_int(-e);
                     sfw[0] |= static_cast<uint32_t>(e + 127) << (8 * k);

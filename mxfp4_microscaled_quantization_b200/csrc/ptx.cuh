@@ -490,6 +490,35 @@ __device__ __forceinline__ float e4m3_decode(uint32_t b) {
     return f;
 }
 
+// Block exponent of an MXFP4 block of P from x = log2 of the block's largest
+// exponential (x <= 0; -inf for a block that is all masked), in the log
+// domain: e = sign * floor(sign * x + off) + add, with (sign, off, add) =
+// (-1, log2 Qmax, 0) for a boundary Qmax < 8, i.e. the smallest e with
+// 2^x <= Qmax * 2^e, and (+1, 0, -2) for OCP, i.e. floor(x) - 2.  Clamped to
+// [-127, ...]; |z| is clamped first so the round-down add stays exact.
+__device__ __forceinline__ int p_block_exponent(float x, float e_sign, float e_off, int e_add) {
+    float z = fmaf(e_sign, x, e_off);
+    z = fminf(fmaxf(z, -250.f), 250.f);
+    const int fl = static_cast<int>(__float_as_uint(__fadd_rd(z, 12582912.f)) - 0x4B400000u);
+    const int e = (e_sign > 0.f ? fl : -fl) + e_add;
+    return e < -127 ? -127 : e;
+}
+
+// NVFP4 block of P from x = log2 of the block's largest exponential: the E4M3
+// scale sb = E4M3(2^x * 448) and the log2 of the element factor 2688 / sb
+// (0 when sb is 0).  log2(sb) is its fp32 exponent plus lg2.approx of its
+// significand, so lg2.approx only sees [1, 2), where its absolute error is
+// smallest.
+__device__ __forceinline__ uint32_t nv_p_block_scale(float x, float& sbv, float& log2_factor) {
+    const uint32_t sb = e4m3_encode_sat(ex2_approx(x) * 448.f);
+    sbv = e4m3_decode(sb);
+    const uint32_t bits = __float_as_uint(sbv);
+    const float l2 = static_cast<float>(static_cast<int>(bits >> 23) - 127) +
+                     lg2_approx(__uint_as_float((bits & 0x7FFFFFu) | 0x3F800000u));
+    log2_factor = sbv > 0.f ? 11.392317422778761f - l2 : 0.f;  // log2(2688) - log2(sb)
+    return sb;
+}
+
 // Block exponent from the bfloat16 bit pattern of a block maximum (>= 0)
 // under a scale boundary Qmax in (4, 8]: the smallest e with amax <= Qmax * 2^e
 // is floor(log2 amax) - 2, plus one when the significand exceeds Qmax / 4,

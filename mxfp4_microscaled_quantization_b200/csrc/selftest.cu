@@ -1,10 +1,19 @@
-// selftest.cu -- mxattn_wait_selftest: drives the attention kernel's bounded
-// mbarrier wait to its time limit on purpose, so that a caller can check that
-// a wait which is never satisfied ends, reports MXATTN_ERR_TIMEOUT and leaves
-// the CUDA context usable.  Nothing here faults or traps: the kernel waits on
-// an mbarrier that nobody arrives at (unless asked to arrive) and returns.
+// selftest.cu -- self-tests of pieces of the attention kernel.
+//
+// mxattn_wait_selftest drives the kernel's bounded mbarrier wait to its time
+// limit on purpose, so that a caller can check that a wait which is never
+// satisfied ends, reports MXATTN_ERR_TIMEOUT and leaves the CUDA context
+// usable.  Nothing here faults or traps: the kernel waits on an mbarrier that
+// nobody arrives at (unless asked to arrive) and returns.
+//
+// mxattn_p_selftest runs the softmax's decisions on P -- E2M1 codes of the
+// exponentials on each of the three exponential paths, the MXFP4 block
+// exponent and the NVFP4 block scale -- on caller inputs, through the same
+// device functions the attention kernel uses, so they can be compared with
+// the CPU oracle directly.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 
 #include "mxattn.h"
@@ -42,8 +51,70 @@ __global__ void __launch_bounds__(32) wait_selftest_kernel(int arrive, uint64_t 
     }
 }
 
+// The softmax's P decisions on a list of inputs, through the same device
+// functions the attention kernel calls (8 inputs per thread, grid-stride).
+//   path 0/1/2: in = w, out = E2M1 code of 2^w by ex2.approx / the FMA-pipe
+//               code-only stand-in / the FMA-pipe degree-5 exponential, each
+//               followed by cvt.rn.satfinite.e2m1x2;
+//   path 3:     in = x (log2 of a block's largest exponential), out = the
+//               MXFP4 block exponent for the scale boundary (e_sign, e_off, e_add);
+//   path 4:     in = x, out = the NVFP4 block scale byte (E4M3 of 2^x * 448).
+__global__ void __launch_bounds__(256) p_selftest_kernel(int path, const float* __restrict__ in, int64_t n8,
+                                                         float e_sign, float e_off, int e_add,
+                                                         int32_t* __restrict__ out) {
+    for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < n8;
+         g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = in[8 * g + i];
+        if (path <= 2) {
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+                if (path == 0) {
+                    f[i] = ex2_approx(v[i]);
+                    f[i + 1] = ex2_approx(v[i + 1]);
+                } else if (path == 1) {
+                    exp2_code_x2(v[i], v[i + 1], f[i], f[i + 1]);
+                } else {
+                    exp2_fma_x2(v[i], v[i + 1], f[i], f[i + 1]);
+                }
+            }
+            const uint32_t codes = pack_e2m1x8(f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) out[8 * g + i] = static_cast<int32_t>((codes >> (4 * i)) & 0xFu);
+        } else if (path == 3) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) out[8 * g + i] = p_block_exponent(v[i], e_sign, e_off, e_add);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float sbv, lf;
+                out[8 * g + i] = static_cast<int32_t>(nv_p_block_scale(v[i], sbv, lf));
+            }
+        }
+    }
+}
+
 }  // namespace
 }  // namespace mxattn
+
+MXATTN_API mxattn_status mxattn_p_selftest(int path, const float* in, int64_t n, float qmax, int32_t* out,
+                                           mxattn_stream_t stream) {
+    if (path < 0 || path > 4 || n < 0 || n % 8 != 0) return MXATTN_ERR_INVALID;
+    if (path == 3 && !(qmax > 4.f && qmax <= 8.f)) return MXATTN_ERR_INVALID;
+    if (n == 0) return MXATTN_OK;
+    if (in == nullptr || out == nullptr || (reinterpret_cast<uintptr_t>(in) & 3u) || (reinterpret_cast<uintptr_t>(out) & 3u))
+        return MXATTN_ERR_INVALID;
+    const bool ocp = qmax >= 8.f;
+    const float e_sign = ocp ? 1.f : -1.f;
+    const float e_off = ocp ? 0.f : static_cast<float>(std::log2(static_cast<double>(qmax)));
+    const int64_t n8 = n / 8;
+    const int grid = static_cast<int>(n8 / 256 + 1 < 4096 ? n8 / 256 + 1 : 4096);
+    mxattn::p_selftest_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(path, in, n8, e_sign, e_off,
+                                                                                         ocp ? -2 : 0, out);
+    return cudaGetLastError() == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
+}
 
 MXATTN_API mxattn_status mxattn_wait_selftest(int arrive, unsigned timeout_us, unsigned* out, mxattn_stream_t stream) {
     if (out == nullptr || timeout_us == 0 || timeout_us > 1000000u) return MXATTN_ERR_INVALID;

@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.mxattn_workspace_status.restype = i32
         L.mxattn_wait_selftest.argtypes = [i32, ctypes.c_uint, P, P]
         L.mxattn_wait_selftest.restype = i32
+        L.mxattn_p_selftest.argtypes = [i32, P, i64, f32, P, P]
+        L.mxattn_p_selftest.restype = i32
         L.mxattn_nvfp4_quantize.argtypes = [P, i64, i64, P, P, P, P]
         L.mxattn_nvfp4_quantize.restype = i32
         L.mxattn_nvfp4_workspace_size.argtypes = [i32, i32, i32, i32]
@@ -286,6 +288,16 @@ def mxattn_wait_selftest(arrive: bool, timeout_us: int, out: torch.Tensor, strea
         raise MxattnError(1, "out must be a contiguous int32 tensor with 3 elements")
     _check(lib().mxattn_wait_selftest(int(bool(arrive)), int(timeout_us), _cuda(out, "out"), _stream(stream)),
            "mxattn_wait_selftest")
+
+
+def mxattn_p_selftest(path: int, x: torch.Tensor, qmax: float = 7.25, out=None, stream=None) -> torch.Tensor:
+    """The attention kernel's P decisions on inputs x (fp32, numel % 8 == 0):
+    E2M1 codes of 2^x (paths 0-2), MXFP4 block exponents (3), NVFP4 block scales (4)."""
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.int32, device=x.device)
+    _check(lib().mxattn_p_selftest(int(path), _cuda(x, "x", torch.float32), x.numel(), float(qmax),
+                                   _cuda(out, "out", torch.int32), _stream(stream)), "mxattn_p_selftest")
+    return out
 
 
 def mxattn_status_string(status: int) -> str:

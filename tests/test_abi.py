@@ -132,3 +132,14 @@ def test_nvfp4_entry_points_reject_bad_arguments_before_launching(L):
     assert L.mxattn_nvfp4_prepare(fake, fake, fake, 1, 1, 256, 128, fake, mx.mxattn_workspace_size(1, 1, 256, 128),
                                   None) == 1
     assert L.mxattn_nvfp4_attend(1, 1, 256, 64, 64, 1, f(0.0), fake, fake, ws_ok - 1, None) == 1
+
+
+def test_p_selftest_rejects_bad_arguments_before_launching(L):
+    fake = _p(1 << 20)
+    f = ctypes.c_float
+    assert L.mxattn_p_selftest(5, fake, 8, f(7.25), fake, None) == 1    # unknown path
+    assert L.mxattn_p_selftest(0, fake, 12, f(7.25), fake, None) == 1   # n % 8 != 0
+    assert L.mxattn_p_selftest(3, fake, 8, f(9.0), fake, None) == 1     # boundary outside (4, 8]
+    assert L.mxattn_p_selftest(0, None, 8, f(7.25), fake, None) == 1    # null input
+    assert L.mxattn_p_selftest(0, _p((1 << 20) + 2), 8, f(7.25), fake, None) == 1  # misaligned
+    assert L.mxattn_p_selftest(1, None, 0, f(7.25), None, None) == 0    # empty is a no-op
