@@ -5,14 +5,20 @@ The compute runs in ``libmxattn.so`` (CUDA kernels for sm_100a); this package
 only marshals arguments.  Importing it does not load the library; the first
 call does, and fails loudly if the library was not built.
 """
-from . import workloads  # noqa: F401
+from . import ulysses, workloads  # noqa: F401
 from .mxattn import (  # noqa: F401
     MxattnError,
     attention_from_host,
     declared_symbols,
     mxattn_attend,
     mxattn_forward,
+    mxattn_forward_noalloc,
     mxattn_forward_quantized,
+    mxattn_nvfp4_attend,
+    mxattn_nvfp4_forward,
+    mxattn_nvfp4_prepare,
+    mxattn_nvfp4_quantize,
+    mxattn_p_selftest,
     mxattn_prepare,
     mxattn_quantize,
     mxattn_quantize_vt,
@@ -20,6 +26,9 @@ from .mxattn import (  # noqa: F401
     mxattn_wait_selftest,
     mxattn_workspace_size,
     mxattn_workspace_status,
+    new_nvfp4_workspace,
     new_workspace,
+    nvfp4_workspace_layout,
+    nvfp4_workspace_size,
     workspace_layout,
 )
