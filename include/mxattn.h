@@ -310,7 +310,9 @@ mxattn_status mxattn_nvfp4_attend(int B, int H, int N, int d, int kv_tile, int p
  *     rounded by cvt.rn.satfinite.e2m1x2;
  *   path 3: in = x (log2 of a block's largest exponential, <= 0), out = the
  *     MXFP4 block exponent e for the scale boundary qmax in (4, 8] (8 = OCP);
- *   path 4: in = x, out = the NVFP4 block scale byte E4M3(2^x * 448).
+ *   path 4: in = x, out = the NVFP4 block scale byte E4M3(2^x * 448);
+ *   path 5: in = v, out = E2M1 code (0..15) of v by cvt.rn.satfinite.e2m1x2
+ *     alone (the rounding step every path ends with).
  *   in: device fp32 [n], out: device i32 [n], both 4-byte aligned; n % 8 == 0.
  * Errors: MXATTN_ERR_INVALID (path, n, qmax for path 3, null or misaligned
  * pointers), MXATTN_ERR_CUDA (launch failed).  Asynchronous on `stream`.

@@ -58,7 +58,8 @@ __global__ void __launch_bounds__(32) wait_selftest_kernel(int arrive, uint64_t 
 //               followed by cvt.rn.satfinite.e2m1x2;
 //   path 3:     in = x (log2 of a block's largest exponential), out = the
 //               MXFP4 block exponent for the scale boundary (e_sign, e_off, e_add);
-//   path 4:     in = x, out = the NVFP4 block scale byte (E4M3 of 2^x * 448).
+//   path 4:     in = x, out = the NVFP4 block scale byte (E4M3 of 2^x * 448);
+//   path 5:     in = v, out = E2M1 code of v itself (the rounding step alone).
 __global__ void __launch_bounds__(256) p_selftest_kernel(int path, const float* __restrict__ in, int64_t n8,
                                                          float e_sign, float e_off, int e_add,
                                                          int32_t* __restrict__ out) {
@@ -67,11 +68,14 @@ __global__ void __launch_bounds__(256) p_selftest_kernel(int path, const float* 
         float v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = in[8 * g + i];
-        if (path <= 2) {
+        if (path <= 2 || path == 5) {
             float f[8];
 #pragma unroll
             for (int i = 0; i < 8; i += 2) {
-                if (path == 0) {
+                if (path == 5) {
+                    f[i] = v[i];
+                    f[i + 1] = v[i + 1];
+                } else if (path == 0) {
                     f[i] = ex2_approx(v[i]);
                     f[i + 1] = ex2_approx(v[i + 1]);
                 } else if (path == 1) {
@@ -101,7 +105,7 @@ __global__ void __launch_bounds__(256) p_selftest_kernel(int path, const float* 
 
 MXATTN_API mxattn_status mxattn_p_selftest(int path, const float* in, int64_t n, float qmax, int32_t* out,
                                            mxattn_stream_t stream) {
-    if (path < 0 || path > 4 || n < 0 || n % 8 != 0) return MXATTN_ERR_INVALID;
+    if (path < 0 || path > 5 || n < 0 || n % 8 != 0) return MXATTN_ERR_INVALID;
     if (path == 3 && !(qmax > 4.f && qmax <= 8.f)) return MXATTN_ERR_INVALID;
     if (n == 0) return MXATTN_OK;
     if (in == nullptr || out == nullptr || (reinterpret_cast<uintptr_t>(in) & 3u) || (reinterpret_cast<uintptr_t>(out) & 3u))

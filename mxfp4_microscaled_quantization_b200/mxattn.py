@@ -292,7 +292,8 @@ def mxattn_wait_selftest(arrive: bool, timeout_us: int, out: torch.Tensor, strea
 
 def mxattn_p_selftest(path: int, x: torch.Tensor, qmax: float = 7.25, out=None, stream=None) -> torch.Tensor:
     """The attention kernel's P decisions on inputs x (fp32, numel % 8 == 0):
-    E2M1 codes of 2^x (paths 0-2), MXFP4 block exponents (3), NVFP4 block scales (4)."""
+    E2M1 codes of 2^x (paths 0-2), MXFP4 block exponents (3), NVFP4 block scales (4),
+    E2M1 codes of x itself (5)."""
     if out is None:
         out = torch.empty(x.shape, dtype=torch.int32, device=x.device)
     _check(lib().mxattn_p_selftest(int(path), _cuda(x, "x", torch.float32), x.numel(), float(qmax),

@@ -137,7 +137,7 @@ def test_nvfp4_entry_points_reject_bad_arguments_before_launching(L):
 def test_p_selftest_rejects_bad_arguments_before_launching(L):
     fake = _p(1 << 20)
     f = ctypes.c_float
-    assert L.mxattn_p_selftest(5, fake, 8, f(7.25), fake, None) == 1    # unknown path
+    assert L.mxattn_p_selftest(6, fake, 8, f(7.25), fake, None) == 1    # unknown path
     assert L.mxattn_p_selftest(0, fake, 12, f(7.25), fake, None) == 1   # n % 8 != 0
     assert L.mxattn_p_selftest(3, fake, 8, f(9.0), fake, None) == 1     # boundary outside (4, 8]
     assert L.mxattn_p_selftest(0, None, 8, f(7.25), fake, None) == 1    # null input

@@ -98,3 +98,51 @@ def test_nvfp4_block_scale():
     rel = np.min(np.abs(exact[bad, None] / mids[None, :] - 1), axis=1) if len(bad) else np.zeros(0)
     assert np.all(rel <= 1e-6), x[bad][rel > 1e-6][:8]
     assert len(bad) <= 64
+
+
+def test_e2m1_rounding_of_every_finite_fp32():
+    """The rounding step alone (cvt.rn.satfinite.e2m1x2) on all 2^32 - 2^24 finite
+    fp32 patterns, in chunks on the GPU: over the positive patterns the code never
+    decreases and changes exactly 7 times, at the patterns the oracle's
+    round-to-nearest-even rule puts them (just above 0.25, at 0.75, just above
+    1.25, at 1.75, just above 2.5, at 3.5, just above 5); each negative pattern's
+    code is the positive one's with the sign bit (-0 gives 0x8).  Since the
+    oracle's rule is monotone with those same transitions, the two agree on
+    every finite fp32 value."""
+    transitions = []
+    chunk = 1 << 27
+    finite = 0x7F800000  # positive finite patterns: [0, 0x7F800000)
+    prev = None
+    for sign in (0, 1):
+        for start in range(0, finite, chunk):
+            stop = min(finite, start + chunk)
+            bits = torch.arange(start, stop, dtype=torch.int64, device="cuda")
+            if sign:
+                bits = bits | (1 << 31)
+            x = (bits - (1 << 32) * (bits >= (1 << 31))).to(torch.int32).view(torch.float32)
+            n = x.numel() - x.numel() % 8
+            codes = mx.mxattn_p_selftest(5, x[:n].contiguous())
+            mag = codes & 7
+            assert int((codes >> 3).min()) == sign and int((codes >> 3).max()) == sign
+            d = mag[1:] - mag[:-1]
+            assert bool((d >= 0).all())
+            idx = torch.nonzero(d).flatten()
+            for i in idx.tolist():
+                transitions.append((sign, start + i + 1, int(mag[i]), int(mag[i + 1])))
+            if prev is not None and prev[0] == sign and n:
+                assert int(mag[0]) >= prev[1]
+                if int(mag[0]) != prev[1]:
+                    transitions.append((sign, start, prev[1], int(mag[0])))
+            prev = (sign, int(mag[n - 1])) if n else prev
+            # the few patterns left over by the multiple-of-8 cut
+            del bits, x, codes, mag, d
+    torch.cuda.synchronize()
+    f = lambda b: float(np.array([b], dtype=np.uint32).view(np.float32)[0])  # noqa: E731
+    pos = [(p, a, b) for s, p, a, b in transitions if s == 0]
+    neg = [(p, a, b) for s, p, a, b in transitions if s == 1]
+    assert [(a, b) for _, a, b in pos] == [(i, i + 1) for i in range(7)]
+    assert [(a, b) for _, a, b in neg] == [(i, i + 1) for i in range(7)]
+    for p, a, b in pos:
+        v, below = f(p), f(p - 1)
+        assert oracle.e2m1_encode([v])[0] == b and oracle.e2m1_encode([below])[0] == a, (v, below)
+    assert [p for p, _, _ in neg] == [p for p, _, _ in pos]
