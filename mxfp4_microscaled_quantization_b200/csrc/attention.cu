@@ -14,10 +14,13 @@
 // threads, three warpgroups; setmaxnreg gives the two softmax warpgroups 224
 // registers per thread and the third 56):
 //   warps 0-3 / 4-7    softmax for tile A / B, one thread per query row (=
-//                      TMEM lane): running max, exp2 on the MUFU with packed
-//                      f32x2 FMAs, per-32-column block exponent (UOS/OCP),
-//                      E2M1 packing of P into shared memory, O rescale in TMEM
-//                      when the max moved, and the final O / l.
+//                      TMEM lane): running max, per-32-column block exponent
+//                      (UOS/OCP) in the log domain, the exponentials with the
+//                      block scale folded into one packed f32x2 FMA -- 9 of 16
+//                      pairs on the MUFU, 7 on the FMA pipe (a code-only
+//                      stand-in for 2^w under PNQ) -- E2M1 packing of P into
+//                      shared memory, O rescale in TMEM when the max moved,
+//                      and the final O / l.
 //   warp 8 (one lane)  TMA producer: both Q tiles + scales once, then K and
 //                      V^T tiles (+ scales) into a kStages-deep ring.
 //   warp 9 (one lane)  MMA issuer: tcgen05.cp of E8M0 scales into TMEM and
@@ -30,6 +33,11 @@
 // sum_j q_j -- exactly the quantized values that multiply V -- and is
 // rescaled together with O.  Without PNQ the row sum of the unquantized
 // exponentials is kept in a register.
+//
+// The same template with NV = true is the NVFP4 comparison variant:
+// tcgen05.mma kind::mxf4nvf4 block16 with E4M3 scale factors, P in blocks of
+// 16 keys with E4M3 scales, and per-(batch, head) second-level scales folded
+// into the softmax scale and the epilogue.
 //
 // Every mbarrier wait is bounded (kTimeoutNs); a wait that gives up records
 // MXATTN_ERR_TIMEOUT in the status word, raises a CTA-wide abort flag, and
