@@ -143,3 +143,28 @@ def test_p_selftest_rejects_bad_arguments_before_launching(L):
     assert L.mxattn_p_selftest(0, None, 8, f(7.25), fake, None) == 1    # null input
     assert L.mxattn_p_selftest(0, _p((1 << 20) + 2), 8, f(7.25), fake, None) == 1  # misaligned
     assert L.mxattn_p_selftest(1, None, 0, f(7.25), None, None) == 0    # empty is a no-op
+
+
+def test_header_compiles_as_c_and_links(L, tmp_path):
+    """include/mxattn.h is plain C (C99, no torch or CUDA headers needed): a C program
+    includes it, links against libmxattn.so and calls the host-only entry points."""
+    import os
+
+    src = tmp_path / "abi.c"
+    src.write_text(
+        "#include <stdio.h>\n#include \"mxattn.h\"\n"
+        "int main(void) {\n"
+        "  size_t ws = mxattn_workspace_size(1, 40, 32760, 128);\n"
+        "  size_t nv = mxattn_nvfp4_workspace_size(1, 40, 32760, 128);\n"
+        "  mxattn_status st = mxattn_quantize(0, 4, 48, MXATTN_RULE_UOS, 0, 0, 0);\n"
+        "  printf(\"%zu %zu %d %s\\n\", ws, nv, (int)st, mxattn_status_string(st));\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(mx.LIB_PATH)
+    inc = os.path.join(os.path.dirname(libdir), "include")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", inc, str(src), "-o", str(exe), f"-L{libdir}",
+                    "-l:libmxattn.so", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert int(out[0]) == mx.mxattn_workspace_size(1, 40, 32760, 128)
+    assert int(out[1]) == mx.nvfp4_workspace_size(1, 40, 32760, 128)
+    assert out[2] == "1" and " ".join(out[3:]) == mx.status_string(1)
