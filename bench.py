@@ -39,7 +39,9 @@ WORKLOAD = wl.WORKLOADS["video_dit"]
 FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor ratio (9 : 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ATTN_PROFILE = os.path.join(ROOT, "profiles", "attention_video_dit.md")
-ATTN_SOURCE = os.path.join(ROOT, "mxfp4_microscaled_quantization_b200", "csrc", "attention.cu")
+# the attention kernel's source: attention.cu and the device functions it inlines from ptx.cuh
+ATTN_SOURCES = tuple(os.path.join(ROOT, "mxfp4_microscaled_quantization_b200", "csrc", f)
+                     for f in ("attention.cu", "ptx.cuh"))
 
 
 def config_dict(w=WORKLOAD):
@@ -62,17 +64,21 @@ def load_peaks():
 
 def profiled_traffic():
     """Per-launch DRAM bytes of the attention kernel from the committed ncu
-    summary, if it was taken on the current attention.cu; else None."""
+    summary, if it was taken on the current kernel source (attention.cu then
+    ptx.cuh, hashed together); else None."""
     try:
         with open(ATTN_PROFILE) as f:
             text = f.read()
-        with open(ATTN_SOURCE, "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()[:16]
+        h = hashlib.sha256()
+        for path in ATTN_SOURCES:
+            with open(path, "rb") as f:
+                h.update(f.read())
+        digest = h.hexdigest()[:16]
     except OSError:
         return None
     src = [ln for ln in text.splitlines() if ln.startswith("source_sha256_16:")]
     tr = [ln for ln in text.splitlines() if ln.startswith("dram_bytes_per_full_launch:")]
-    if not src or not tr or src[0].split(":", 1)[1].strip() != digest:
+    if not src or not tr or src[0].split(":", 1)[1].split()[0] != digest:
         return None
     return float(tr[0].split(":", 1)[1].strip())
 
@@ -227,10 +233,10 @@ def quantize_sweep_point(torch, mx, peaks, peak_kind, log2n=30, iters=10):
     return out
 
 
-# MUFU exponentials per S element in mxattn_fwd_kernel with PNQ: 9 of every 16
-# pairs on the MUFU (ex2.approx), 7 on the FMA pipe; plus the rescale factor,
+# MUFU exponentials per S element in mxattn_fwd_kernel with PNQ: 8 of every 16
+# pairs on the MUFU (ex2.approx), 8 on the FMA pipe; plus the rescale factor,
 # one per row and 128-column key tile.  Block exponents take no exponential.
-MUFU_EX2_PER_ELEMENT = 9.0 / 16 + 1.0 / 128
+MUFU_EX2_PER_ELEMENT = 8.0 / 16 + 1.0 / 128
 
 
 def mufu_roofline(w, attn_ms, clocks, sms=148, ex2_per_clk_per_sm=16):

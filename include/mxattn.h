@@ -305,9 +305,10 @@ mxattn_status mxattn_nvfp4_attend(int B, int H, int N, int d, int kv_tile, int p
  * paper has no counterpart).  Runs, on n inputs, the device functions the
  * attention kernel uses for P, so they can be compared with a reference:
  *   path 0, 1, 2: in = w (fp32), out = E2M1 code (0..15) of 2^w computed by
- *     ex2.approx (0), by the FMA-pipe code-only stand-in used with PNQ (1),
- *     or by the FMA-pipe degree-5 exponential used without PNQ (2), each
- *     rounded by cvt.rn.satfinite.e2m1x2;
+ *     ex2.approx (0), by the FMA-pipe code-only stand-in used with PNQ (1;
+ *     its input map u = sat((w + 2) / 8) included), or by the FMA-pipe
+ *     degree-5 exponential used without PNQ (2), each rounded by
+ *     cvt.rn.satfinite.e2m1x2;
  *   path 3: in = x (log2 of a block's largest exponential, <= 0), out = the
  *     MXFP4 block exponent e for the scale boundary qmax in (4, 8] (8 = OCP);
  *   path 4: in = x, out = the NVFP4 block scale byte E4M3(2^x * 448);

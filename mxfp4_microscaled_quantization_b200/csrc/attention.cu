@@ -16,9 +16,10 @@
 //   warps 0-3 / 4-7    softmax for tile A / B, one thread per query row (=
 //                      TMEM lane): running max, per-32-column block exponent
 //                      (UOS/OCP) in the log domain, the exponentials with the
-//                      block scale folded into one packed f32x2 FMA -- 9 of 16
-//                      pairs on the MUFU, 7 on the FMA pipe (a code-only
-//                      stand-in for 2^w under PNQ) -- E2M1 packing of P into
+//                      block scale folded into the bias of one FMA -- under
+//                      PNQ 8 of 16 pairs on the MUFU and 8 on the FMA pipe (a
+//                      code-only stand-in for 2^w), without PNQ 10 and 6 (a
+//                      full polynomial exponential) -- E2M1 packing of P into
 //                      shared memory, O rescale in TMEM when the max moved,
 //                      and the final O / l.
 //   warp 8 (one lane)  TMA producer: both Q tiles + scales once, then K and
@@ -103,11 +104,11 @@ struct Cfg {
     static constexpr int kSfSlots = NV ? 2 : kStages;
     static constexpr int kOCols = D + 16;
     // Of the 16 exponential pairs of a 32-column block, this many go to the FMA
-    // pipe instead of the MUFU: 7 with PNQ (the code-only stand-in for 2^w,
-    // exp2_code_x2), 6 without (the full polynomial, exp2_fma_x2); pair q is
+    // pipe instead of the MUFU: 8 with PNQ (the code-only stand-in for 2^w,
+    // exp2_code_sat_x2), 6 without (the full polynomial, exp2_fma_x2); pair q is
     // one of them when (q * n) mod 16 < n, which spreads them evenly.
     __host__ __device__ static constexpr bool fma_pair(int q, bool pnq) {
-        const int n = pnq ? 7 : 6;  // measured best for both formats (NVFP4: 6, 7 and 8 tie with PNQ)
+        const int n = pnq ? 8 : 6;  // measured best for both formats
         return (q * n) % 16 < n;
     }
 
@@ -473,6 +474,7 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
             kq = p.kq / (Gq * Gk);
             o_unit = __fmul_rn(6.f, p.gs[2 * p.BH + bh]);
         }
+        const float kq8 = 0.125f * kq;  // exact: the stand-in's map of w onto [0, 1] scales by 1/8
         const float e_sign = p.e_sign;
         const float e_off = p.e_off;
         const int e_add = p.e_add;
@@ -522,17 +524,21 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
             float lsum = 0.f;
             // Per block of P: `nbias[k]` turns s * kq into the log2 of the element as it
             // enters the E2M1 rounding, `back[k]` brings a rounded value back to exp(s - m_new).
-            float nbias[NBM], back[NBM];
+            // `nb8[k]` = (nbias[k] + 2) / 8 is the same bias for the code-only stand-in
+            // (exp2_code_sat_x2), formed with one rounding like nbias.
+            float nbias[NBM], nb8[NBM], back[NBM];
             if constexpr (NV) {
                 // NVFP4 P (blocks of 16 keys): scale sb = E4M3(pmax * 448) with pmax the block's
                 // largest exponential, element = exp(s - m_new) * 2688 / sb.  A block whose scale
                 // rounds to 0 holds values below 2.3e-6 and is left unscaled (all its codes are 0).
 #pragma unroll
                 for (int k = 0; k < NBM; ++k) {
-                    float sbv, lf;
-                    const uint32_t sb = nv_p_block_scale((bm[k] - m_new) * kq, sbv, lf);
-                    nbias[k] = fmaf(-m_new, kq, lf);
-                    back[k] = sbv > 0.f ? sbv * (1.f / 2688.f) : 1.f;
+                    float sbv, l2;
+                    const uint32_t sb = nv_p_block_scale((bm[k] - m_new) * kq, sbv, l2);
+                    const bool scaled = sbv > 0.f;
+                    nbias[k] = fmaf(-m_new, kq, scaled ? 11.392317422778761f - l2 : 0.f);  // log2(2688 / sb)
+                    if constexpr (PNQ) nb8[k] = 0.125f * fmaf(-m_new, kq, scaled ? 13.392317422778761f - l2 : 2.f);
+                    back[k] = scaled ? sbv * (1.f / 2688.f) : 1.f;
                     sfw[k / 4] |= sb << (8 * (k % 4));
                 }
             } else {
@@ -545,6 +551,7 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
                     // the OCP boundary at integer x is decided exactly there.
                     const int e = p_block_exponent((bm[k] - m_new) * kq, e_sign, e_off, e_add);
                     nbias[k] = -fmaf(m_new, kq, static_cast<float>(e));
+                    if constexpr (PNQ) nb8[k] = -0.125f * fmaf(m_new, kq, static_cast<float>(e - 2));
                     back[k] = exp2_neg_int(-e);
                     sfw[0] |= static_cast<uint32_t>(e + 127) << (8 * k);
                 }
@@ -557,13 +564,14 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 8; i += 2) {
                     float w0, w1;
-                    ffma2_bcast(w0, w1, sv[8 * gg + i], sv[8 * gg + i + 1], kq, nbias[k]);
                     if (!C::fma_pair(4 * (gg % 4) + i / 2, PNQ)) {  // MUFU
+                        ffma2_bcast(w0, w1, sv[8 * gg + i], sv[8 * gg + i + 1], kq, nbias[k]);
                         f[i] = ex2_approx(w0);
                         f[i + 1] = ex2_approx(w1);
                     } else if constexpr (PNQ) {  // FMA pipe: only the E2M1 code is kept
-                        exp2_code_x2(w0, w1, f[i], f[i + 1]);
+                        exp2_code_sat_x2(sv[8 * gg + i], sv[8 * gg + i + 1], kq8, nb8[k], f[i], f[i + 1]);
                     } else {                     // FMA pipe: the value enters the row sum
+                        ffma2_bcast(w0, w1, sv[8 * gg + i], sv[8 * gg + i + 1], kq, nbias[k]);
                         exp2_fma_x2(w0, w1, f[i], f[i + 1]);
                     }
                 }

@@ -380,42 +380,47 @@ __device__ __forceinline__ void exp2_fma_x2(float w0, float w1, float& v0, float
 }
 
 // A stand-in for 2^w whose E2M1 code (cvt.rn.satfinite.e2m1x2) equals the
-// code of 2^w, for two values on the FMA pipe.  The code of 2^w depends only
-// on where w falls against the E2M1 rounding points: the integer part
-// n = floor(w) picks the binade and the fraction f = w - n decides the
-// mantissa, whose rounding points 1.25, 1.5 and 1.75 are crossed at
-// f = log2(1.25), log2(1.5), log2(1.75).  z(f) = 1 + f (c1 + f (c2 + f c3))
-// is the cubic that passes through those three points and z(0) = 1 exactly
-// (coefficients from csrc/exp2_code_fit.py), is increasing on [0, 1) and stays
-// below 2, so 2^n * z(f) falls on the same side of every rounding point as
-// 2^w (up to fp32 rounding, a few ulp of f, as for ex2.approx).  Its value is
-// NOT 2^w (up to 7.7e-4 off between the points): use it only where nothing
-// but the code is kept.  Inputs are clamped at -8 (every w < -2 has code 0)
-// so the exponent field stays normal.
-__device__ __forceinline__ void exp2_code_x2(float w0, float w1, float& v0, float& v1) {
-    w0 = fmaxf(w0, -8.f);
-    w1 = fmaxf(w1, -8.f);
-    uint32_t p0, p1, t0, t1;
-    asm("{\n\t.reg .b64 w, t, n, f, p, c;\n\t"
-        "mov.b64 w, {%4, %5};\n\t"
+// code of 2^w, for two values on the FMA pipe, with w = s * k + b given as
+// u = sat(s * k8 + b8), k8 = k / 8, b8 = (b + 2) / 8: the saturating FMA maps
+// w in [-2, 6] onto u in [0, 1] and clamps everything outside (w <= -2, every
+// value whose code is 0, gives u = 0; -inf and NaN too).  The code of 2^w only
+// depends on where w falls against the log2 of the seven E2M1 rounding points
+// 0.25, 0.75, 1.25, 1.75, 2.5, 3.5 and 5, so p(u) is the degree-6 polynomial
+// that takes the value t at u = (log2 t + 2) / 8 for each of them (p(0) = 0.25
+// exactly, so the tie at 2^-2 rounds to 0 like the exact value) and increases
+// on [0, 1] (p(1) = 59.4 > 5).  Coefficients from csrc/exp2_code_fit.py.  p
+// lands on the same side of every rounding point as 2^w except within fp32
+// rounding of the crossing (a few ulp of w + 2), as for ex2.approx.  Its value
+// is NOT 2^w (7 % off above the last point): use it only where nothing but
+// the code is kept.  Two scalar FMAs (f32x2 has no saturating form) and six
+// packed ones per pair; no ALU instruction.
+__device__ __forceinline__ void exp2_code_sat_x2(float s0, float s1, float k8, float b8, float& v0, float& v1) {
+    float u0, u1;
+    asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(u0) : "f"(s0), "f"(k8), "f"(b8));
+    asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(u1) : "f"(s1), "f"(k8), "f"(b8));
+    uint32_t p0, p1;
+    asm("{\n\t.reg .b64 u, p, c;\n\t"
+        "mov.b64 u, {%2, %3};\n\t"
+        "mov.b64 p, {%4, %4};\n\t"
+        "mov.b64 c, {%5, %5};\n\t"
+        "fma.rn.f32x2 p, p, u, c;\n\t"
         "mov.b64 c, {%6, %6};\n\t"
-        "add.rm.f32x2 t, w, c;\n\t"      // floor(w) lands in the low mantissa bits of t
-        "sub.rn.f32x2 n, t, c;\n\t"      // n = floor(w)
-        "sub.rn.f32x2 f, w, n;\n\t"      // f in [0, 1]
-        "mov.b64 p, {%10, %10};\n\t"
-        "mov.b64 c, {%9, %9};\n\t"
-        "fma.rn.f32x2 p, p, f, c;\n\t"
-        "mov.b64 c, {%8, %8};\n\t"
-        "fma.rn.f32x2 p, p, f, c;\n\t"
+        "fma.rn.f32x2 p, p, u, c;\n\t"
         "mov.b64 c, {%7, %7};\n\t"
-        "fma.rn.f32x2 p, p, f, c;\n\t"
-        "mov.b64 {%0, %1}, p;\n\t"
-        "mov.b64 {%2, %3}, t;\n\t}"
-        : "=r"(p0), "=r"(p1), "=r"(t0), "=r"(t1)
-        : "f"(w0), "f"(w1), "f"(12582912.0f),  // 1.5 * 2^23
-          "f"(1.0f), "f"(0x1.63d846p-1f), "f"(0x1.d566bep-3f), "f"(0x1.334fcep-4f));
-    v0 = __uint_as_float(p0 + (t0 << 23));
-    v1 = __uint_as_float(p1 + (t1 << 23));
+        "fma.rn.f32x2 p, p, u, c;\n\t"
+        "mov.b64 c, {%8, %8};\n\t"
+        "fma.rn.f32x2 p, p, u, c;\n\t"
+        "mov.b64 c, {%9, %9};\n\t"
+        "fma.rn.f32x2 p, p, u, c;\n\t"
+        "mov.b64 c, {%10, %10};\n\t"
+        "fma.rn.f32x2 p, p, u, c;\n\t"
+        "mov.b64 {%0, %1}, p;\n\t}"
+        : "=r"(p0), "=r"(p1)
+        : "f"(u0), "f"(u1),  // c6 .. c0
+          "f"(0x1.0132fcp+6f), "f"(-0x1.b3010ap+5f), "f"(0x1.6e5d76p+5f), "f"(-0x1.9f6ee0p+1f), "f"(0x1.56cd60p+2f),
+          "f"(0x1.4c45dep+0f), "f"(0x1.000000p-2f));
+    v0 = __uint_as_float(p0);
+    v1 = __uint_as_float(p1);
 }
 
 // ------------------------------------------------------------------ E2M1 / E8M0 helpers
@@ -478,17 +483,15 @@ __device__ __forceinline__ int p_block_exponent(float x, float e_sign, float e_o
 }
 
 // NVFP4 block of P from x = log2 of the block's largest exponential: the E4M3
-// scale sb = E4M3(2^x * 448) and the log2 of the element factor 2688 / sb
-// (0 when sb is 0).  log2(sb) is its fp32 exponent plus lg2.approx of its
-// significand, so lg2.approx only sees [1, 2), where its absolute error is
-// smallest.
-__device__ __forceinline__ uint32_t nv_p_block_scale(float x, float& sbv, float& log2_factor) {
+// scale sb = E4M3(2^x * 448), its value, and log2(sb) (meaningful only when
+// sb > 0).  log2(sb) is its fp32 exponent plus lg2.approx of its significand,
+// so lg2.approx only sees [1, 2), where its absolute error is smallest.
+__device__ __forceinline__ uint32_t nv_p_block_scale(float x, float& sbv, float& log2_sb) {
     const uint32_t sb = e4m3_encode_sat(ex2_approx(x) * 448.f);
     sbv = e4m3_decode(sb);
     const uint32_t bits = __float_as_uint(sbv);
-    const float l2 = static_cast<float>(static_cast<int>(bits >> 23) - 127) +
-                     lg2_approx(__uint_as_float((bits & 0x7FFFFFu) | 0x3F800000u));
-    log2_factor = sbv > 0.f ? 11.392317422778761f - l2 : 0.f;  // log2(2688) - log2(sb)
+    log2_sb = static_cast<float>(static_cast<int>(bits >> 23) - 127) +
+              lg2_approx(__uint_as_float((bits & 0x7FFFFFu) | 0x3F800000u));
     return sb;
 }
 

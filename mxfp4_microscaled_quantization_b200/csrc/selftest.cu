@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(256) p_selftest_kernel(int path, const float* 
                     f[i] = ex2_approx(v[i]);
                     f[i + 1] = ex2_approx(v[i + 1]);
                 } else if (path == 1) {
-                    exp2_code_x2(v[i], v[i + 1], f[i], f[i + 1]);
+                    exp2_code_sat_x2(v[i], v[i + 1], 0.125f, 0.25f, f[i], f[i + 1]);  // u = (w + 2) / 8
                 } else {
                     exp2_fma_x2(v[i], v[i + 1], f[i], f[i + 1]);
                 }
@@ -93,8 +93,8 @@ __global__ void __launch_bounds__(256) p_selftest_kernel(int path, const float* 
         } else {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                float sbv, lf;
-                out[8 * g + i] = static_cast<int32_t>(nv_p_block_scale(v[i], sbv, lf));
+                float sbv, l2;
+                out[8 * g + i] = static_cast<int32_t>(nv_p_block_scale(v[i], sbv, l2));
             }
         }
     }

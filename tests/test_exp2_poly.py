@@ -1,7 +1,16 @@
-"""The FMA-pipe exponential of the attention kernel: its polynomial constants
-are the ones csrc/exp2_poly_fit.py derives (weighted Chebyshev least squares
-of 2^f on [-1/2, 1/2], degree 5), and fp32 Horner evaluation of them stays
-within 2.5e-7 relative error of 2^f, on par with the MUFU ex2.approx."""
+"""The attention kernel's FMA-pipe stand-ins for the MUFU exponential and its
+log-domain block exponent of P, emulated in fp32 on the CPU.
+
+- The exponential used without PNQ: its polynomial constants are the ones
+  csrc/exp2_poly_fit.py derives (weighted Chebyshev least squares of 2^f on
+  [-1/2, 1/2], degree 5), and fp32 Horner evaluation of them stays within
+  2.5e-7 relative error of 2^f, on par with ex2.approx.
+- The code-only stand-in used under PNQ (csrc/exp2_code_fit.py): a degree-6
+  polynomial in u = sat((w + 2) / 8) whose E2M1 code equals that of 2^w except
+  within fp32 rounding of a rounding point.
+- The block exponent of P from the log2 of the block maximum: equal to the
+  scale rule applied to the exact power of two except within fp32 rounding
+  of a boundary."""
 import importlib.util
 import os
 import re
@@ -63,61 +72,64 @@ def _code_fit_module():
 
 
 def _code_kernel_constants():
+    """The stand-in's constants as written in csrc/ptx.cuh (c6 first), returned as c0 .. c6."""
     src = open(os.path.join(PKG, "csrc", "ptx.cuh")).read()
-    body = src[src.index("void exp2_code_x2("):]
+    body = src[src.index("void exp2_code_sat_x2("):]
     body = body[: body.index("v0 = __uint_as_float")]
-    return np.array([float.fromhex(h[:-1]) for h in re.findall(r"0x1\.[0-9a-f]+p[+-]\d+f", body)], dtype=np.float32)
-
-
-def _code_stand_in_f32(w):
-    """exp2_code_x2 emulated in fp32 the way the kernel runs it: clamp at -8,
-    floor via adding 1.5 * 2^23 rounded toward -inf, the cubic in Horner form,
-    2^floor(w) added to the exponent field."""
-    m = _code_fit_module()
-    w = np.maximum(np.asarray(w, dtype=np.float32), np.float32(-8.0))
-    c = np.float64(12582912.0)
-    # fp32 add with round-toward-minus-infinity: the fp64 sum is exact here, floor it to the fp32 grid (ulp 1)
-    t = np.floor(w.astype(np.float64) + c).astype(np.float32)
-    n = (t - np.float32(c)).astype(np.float32)
-    f = (w - n).astype(np.float32)
-    z = m.horner_f32(m.coefficients(), f)
-    bits = (z.view(np.uint32) + (t.view(np.uint32) << np.uint32(23))).astype(np.uint32)
-    return bits.view(np.float32)
+    vals = [float.fromhex(h[:-1]) for h in re.findall(r"-?0x1\.[0-9a-f]+p[+-]\d+f", body)]
+    return np.array(vals[::-1], dtype=np.float32)
 
 
 def test_code_stand_in_uses_the_derived_coefficients():
     np.testing.assert_array_equal(_code_kernel_constants(), _code_fit_module().coefficients())
 
 
-def test_code_stand_in_cubic_shape():
-    """z(0) = 1 exactly, increasing on [0, 1), below 2, and on the right side of
-    each mantissa rounding point everywhere except a few ulp around it."""
+def test_code_stand_in_polynomial_shape():
+    """p(0) = 0.25 exactly, p increasing on [0, 1] in fp32 evaluation, p(1) above
+    the last rounding point 5, and p(u_t) = t to fp32 accuracy at each rounding
+    point t, u_t = (log2 t + 2) / 8 (evaluated here in fp64, apart from the fit)."""
     m = _code_fit_module()
     coef = m.coefficients()
-    f = np.linspace(0.0, 1.0, 400001, dtype=np.float64).astype(np.float32)[:-1]
-    z = m.horner_f32(coef, f).astype(np.float64)
-    assert z[0] == 1.0 and np.all(np.diff(z) >= 0) and z.max() < 2.0
-    assert all(k <= 4 for k in m.crossing_mismatches(coef, ulps=256))
+    u = np.linspace(0.0, 1.0, 400001, dtype=np.float64)
+    p = m.stand_in_f32(coef, (u * 8.0 - 2.0).astype(np.float32)).astype(np.float64)
+    assert p[0] == 0.25 and np.all(np.diff(p) >= 0) and p[-1] > 5.0
+    for t in (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0):
+        uk = (np.log2(t) + 2.0) / 8.0
+        val = sum(float(c) * uk ** i for i, c in enumerate(coef))
+        assert abs(val / t - 1) < 2e-6, (t, val)
+
+
+def test_code_stand_in_crossings_exact_fma():
+    """With every FMA rounded once (exact rational emulation), at most 4 fp32 w
+    within 64 ulp of each crossing log2 t land on the other side of t than 2^w,
+    all within 2e-7 of the crossing."""
+    m = _code_fit_module()
+    for n, far in m.crossing_mismatches(m.coefficients(), ulps=64):
+        assert n <= 4 and far <= 2e-7, (n, far)
 
 
 def test_code_stand_in_gives_the_e2m1_code_of_2_pow_w():
     """The E2M1 code (round to nearest even, saturating) of the stand-in equals
     the code of the exact 2^w for every w on a dense grid over the range the
     kernel feeds it (w <= log2(8) after division by the block scale), apart from
-    w within 4 fp32 ulp of a rounding point's crossing."""
+    w within fp32 rounding of w + 2 (the stand-in's input is u = (w + 2) / 8) of
+    a rounding point's crossing."""
     import oracle
 
+    m = _code_fit_module()
     w = np.concatenate([np.linspace(-130.0, 3.0, 1_000_001), np.arange(-130, 4), [-np.inf]]).astype(np.float32)
-    got = oracle.e2m1_encode(_code_stand_in_f32(w).astype(np.float64))
-    exact = 2.0 ** w.astype(np.float64)
-    ref = oracle.e2m1_encode(exact)
+    got = oracle.e2m1_encode(m.stand_in_f32(m.coefficients(), w).astype(np.float64))
+    ref = oracle.e2m1_encode(2.0 ** w.astype(np.float64))
     bad = np.nonzero(got != ref)[0]
     crossings = np.log2([0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
     for i in bad:
-        assert np.min(np.abs(np.float64(w[i]) - crossings)) <= 4 * np.spacing(np.float32(abs(w[i]) + 1)), w[i]
+        tol = 2 * np.spacing(np.float32(np.float64(w[i]) + 2.0))
+        assert np.min(np.abs(np.float64(w[i]) - crossings)) <= tol, w[i]
     assert len(bad) <= 12
     # every w below -2 is code 0; the tie at 2^-2 rounds to 0 as for the exact value
     assert np.all(got[w < -2] == 0) and got[w == -2][0] == 0
+    # above the last crossing the code is the saturated 6 (code 7)
+    assert np.all(got[w > np.log2(5.0) + 1e-6] == 7)
 
 
 # ---------------------------------------------------------------- block exponent of P in the log domain
