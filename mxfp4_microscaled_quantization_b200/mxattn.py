@@ -316,19 +316,35 @@ def _copy_streams(device):
     return _side_streams[key]
 
 
+def host_groups(BH: int, chunks: int = 16):
+    """Sizes of the (batch, head) groups attention_from_host pipelines by
+    default: `chunks` groups, the first and the last of one slice each (the
+    copy to the device of the first group and the copy back of the last are
+    the only transfers nothing else overlaps), the rest as equal as possible."""
+    if BH <= 0:
+        return []
+    n = max(1, min(int(chunks), BH))
+    if n < 3 or BH < 3:
+        per = -(-BH // n)
+        return [min(per, BH - i) for i in range(0, BH, per)]
+    mid, k = BH - 2, n - 2
+    return [1] + [mid // k + (1 if i < mid % k else 0) for i in range(k)] + [1]
+
+
 def attention_from_host(q_host, k_host, v_host, kv_tile=128, pnq=True, rule="uos", softmax_scale=0.0,
-                        device_buffers=None, out_host=None, stream=None, chunks=16):
+                        device_buffers=None, out_host=None, stream=None, chunks=16, groups=None):
     """End-to-end call with host tensors: q, k, v (pinned host bf16 [B, H, N, d])
     to the device, mxattn_forward, O back into `out_host` (pinned fp32).
 
-    The (batch, head) slices are processed in `chunks` groups, pipelined over
-    three streams: the copy of group i+1 to the device and of group i-1 back to
-    the host overlap the attention of group i (heads are independent, so each
+    The (batch, head) slices are processed in groups (`groups`: their sizes,
+    summing to B*H; default host_groups(B*H, chunks)), pipelined over three
+    streams: the copy of group i+1 to the device and of group i-1 back to the
+    host overlap the attention of group i (heads are independent, so each
     group is one mxattn_forward call on a contiguous slice).  The work is
     ordered on `stream` (default: the current stream): everything, including
     the last copy back, is done when `stream` reaches the point after this call.
     `device_buffers` = (q, k, v, out, workspace) device tensors to reuse; the
-    workspace needs only the size of one group."""
+    workspace needs only the size of the largest group."""
     B, H, N, d = q_host.shape
     BH = B * H
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -340,10 +356,11 @@ def attention_from_host(q_host, k_host, v_host, kv_tile=128, pnq=True, rule="uos
     qd, kd, vd, od, ws = device_buffers
     if out_host is None:
         out_host = torch.empty((B, H, N, d), dtype=torch.float32, pin_memory=True)
-    n_chunks = max(1, min(int(chunks), BH))
-    per = -(-BH // n_chunks)
+    sizes = host_groups(BH, chunks) if groups is None else [int(g) for g in groups]
+    if BH and (sum(sizes) != BH or min(sizes) < 1):
+        raise ValueError(f"groups {sizes} must be positive and sum to B*H = {BH}")
     if ws is None:
-        ws = new_workspace(1, per, N, d, dev)
+        ws = new_workspace(1, max(sizes, default=1), N, d, dev)
     compute = torch.cuda.current_stream(dev) if stream is None else stream
     h2d, d2h = _copy_streams(dev)
     h2d.wait_stream(compute)  # the device buffers may still be in use by earlier work on `stream`
@@ -352,8 +369,10 @@ def attention_from_host(q_host, k_host, v_host, kv_tile=128, pnq=True, rule="uos
     qh, kh, vh, oh = flat(q_host), flat(k_host), flat(v_host), flat(out_host)
     qf, kf, vf, of = flat(qd), flat(kd), flat(vd), flat(od)
     last = None
-    for c0 in range(0, BH, per):
-        sl = slice(c0, min(BH, c0 + per))
+    c0 = 0
+    for size in sizes:
+        sl = slice(c0, c0 + size)
+        c0 += size
         with torch.cuda.stream(h2d):
             qf[sl].copy_(qh[sl], non_blocking=True)
             kf[sl].copy_(kh[sl], non_blocking=True)
@@ -371,7 +390,8 @@ def attention_from_host(q_host, k_host, v_host, kv_tile=128, pnq=True, rule="uos
             oh[sl].copy_(of[sl], non_blocking=True)
             last = torch.cuda.Event()
             last.record(d2h)
-    compute.wait_event(last)
+    if last is not None:
+        compute.wait_event(last)
     return out_host
 
 

@@ -239,13 +239,22 @@ def test_status_string_roundtrip():
     assert math.isfinite(mx.mxattn_workspace_size(1, 40, 32760, 128))
 
 
-@pytest.mark.parametrize("chunks", [1, 3, 8, 100])
-def test_attention_from_host_pipeline_matches_forward(chunks):
-    """The host-to-host call (head groups pipelined over three streams) gives the
-    same O as one mxattn_forward on device tensors, bit for bit."""
+@pytest.mark.parametrize("chunks,groups", [(1, None), (3, None), (8, None), (100, None), (16, [4, 1, 5]), (16, [10])])
+def test_attention_from_host_pipeline_matches_forward(chunks, groups):
+    """The host-to-host call (head groups pipelined over three streams, the
+    default ramped schedule or explicit group sizes) gives the same O as one
+    mxattn_forward on device tensors, bit for bit."""
     Q, K, V = wl.gaussian_qkv(2, 5, 300, 128, seed=31)
     ref, _ = run_forward(Q, K, V, 128, True, "uos")
     host = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()  # noqa: E731
-    out = mx.attention_from_host(host(Q), host(K), host(V), 128, True, "uos", chunks=chunks)
+    out = mx.attention_from_host(host(Q), host(K), host(V), 128, True, "uos", chunks=chunks, groups=groups)
     torch.cuda.current_stream().synchronize()
     np.testing.assert_array_equal(out.numpy().astype(np.float64), ref)
+
+
+def test_attention_from_host_rejects_bad_groups():
+    Q, K, V = wl.gaussian_qkv(1, 3, 64, 64, seed=32)
+    host = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()  # noqa: E731
+    for groups in ([1, 1], [2, 2], [3, 0]):
+        with pytest.raises(ValueError):
+            mx.attention_from_host(host(Q), host(K), host(V), 64, True, "uos", groups=groups)
