@@ -446,23 +446,33 @@ def run_gpu(args, rank, world, local_rank):
     if rank == 0 and not args.quick and not args.no_quantize_sweep and not seq:
         quant = quantize_sweep_point(torch, mx, peaks, peak_kind)
 
-    # The same attention step with the OCP rule and no PNQ (the comparator the
-    # method is measured against): the cost of UOS + PNQ relative to it.
+    # The same attention step under every scale rule x PNQ combination: OCP
+    # without PNQ is the comparator the method is measured against; the two mixed
+    # ones separate the cost of UOS from that of PNQ.
     overhead = None
     if not args.quick and not seq:
-        mx.mxattn_prepare(q, k, v, "ocp", ws)
-        for _ in range(2):
-            mx.mxattn_attend(ws, B, H, N, d, w.kv_tile, False, "ocp", 0.0, out)
-        torch.cuda.synchronize()
-        o0, o1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        o0.record(stream)
-        for _ in range(5):
-            mx.mxattn_attend(ws, B, H, N, d, w.kv_tile, False, "ocp", 0.0, out)
-        o1.record(stream)
-        torch.cuda.synchronize()
-        ocp_ms = max_over_ranks([o0.elapsed_time(o1) / 5], dist, "cuda")[0]
-        overhead = {"ocp_no_pnq_attn_ms": ocp_ms, "uos_pnq_attn_ms": attn_avg_ms,
-                    "uos_pnq_over_ocp": attn_avg_ms / ocp_ms - 1.0}
+        def attend_ms(rule, pnq):
+            mx.mxattn_prepare(q, k, v, rule, ws)
+            for _ in range(2):
+                mx.mxattn_attend(ws, B, H, N, d, w.kv_tile, pnq, rule, 0.0, out)
+            torch.cuda.synchronize()
+            o0, o1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            o0.record(stream)
+            for _ in range(5):
+                mx.mxattn_attend(ws, B, H, N, d, w.kv_tile, pnq, rule, 0.0, out)
+            o1.record(stream)
+            torch.cuda.synchronize()
+            return max_over_ranks([o0.elapsed_time(o1) / 5], dist, "cuda")[0]
+
+        t = {(rule, pnq): attend_ms(rule, pnq) for rule in ("ocp", "uos") for pnq in (False, True)}
+        ocp_ms = t[("ocp", False)]
+        overhead = {"ocp_no_pnq_attn_ms": ocp_ms, "ocp_pnq_attn_ms": t[("ocp", True)],
+                    "uos_no_pnq_attn_ms": t[("uos", False)], "uos_pnq_attn_ms": attn_avg_ms,
+                    "uos_pnq_attn_ms_same_leg": t[("uos", True)],
+                    "uos_pnq_over_ocp": attn_avg_ms / ocp_ms - 1.0,
+                    "uos_over_ocp_with_pnq": t[("uos", True)] / t[("ocp", True)] - 1.0,
+                    "uos_over_ocp_without_pnq": t[("uos", False)] / ocp_ms - 1.0,
+                    "pnq_over_no_pnq_with_uos": t[("uos", True)] / t[("uos", False)] - 1.0}
 
     # The NVFP4 comparison variant (16-element blocks, E4M3 scales, per-head fp32
     # scales) on the same workload and kernel structure, PNQ on.

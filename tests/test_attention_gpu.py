@@ -151,6 +151,30 @@ def test_forward_quantized_matches_forward_bitwise():
     np.testing.assert_array_equal(O2.cpu().numpy(), O1.astype(np.float32))
 
 
+@pytest.mark.parametrize("N,d,T,rule", [(700, 128, 128, "uos"), (129, 64, 64, "ocp"), (300, 64, 128, 6.5),
+                                          (1, 128, 64, "uos"), (1000, 128, 128, "ocp")])
+def test_forward_matches_prepare_attend_and_fills_the_workspace(N, d, T, rule):
+    """mxattn_forward and mxattn_prepare + mxattn_attend give the same O and the
+    same workspace (Q/K/V^T codes and scales) bit for bit, starting from two
+    different fill bytes, so every byte of those regions is written."""
+    Q, K, V = wl.gaussian_qkv(2, 3, N, d, seed=13)
+    q, k, v = _dev(Q), _dev(K), _dev(V)
+    ws1 = mx.new_workspace(2, 3, N, d)
+    ws2 = mx.new_workspace(2, 3, N, d)
+    ws1.fill_(0x5A)  # different fills: a byte either path leaves unwritten shows up as a difference
+    ws2.fill_(0xA5)
+    O1 = mx.mxattn_forward(q, k, v, T, True, rule, 0.0, workspace=ws1)
+    mx.mxattn_prepare(q, k, v, rule, ws2)
+    O2 = torch.empty_like(O1)
+    mx.mxattn_attend(ws2, 2, 3, N, d, T, True, rule, 0.0, O2)
+    torch.cuda.synchronize()
+    assert mx.mxattn_workspace_status(ws1) == 0 and mx.mxattn_workspace_status(ws2) == 0
+    assert torch.equal(O1, O2)
+    for name in ("q_codes", "q_sf", "k_codes", "k_sf", "vt_codes", "vt_sf"):
+        a, b = _region(ws1, name, 2, 3, N, d), _region(ws2, name, 2, 3, N, d)
+        np.testing.assert_array_equal(a, b, err_msg=name)
+
+
 @pytest.mark.parametrize("d,T", [(64, 64), (128, 128), (128, 64)])
 def test_forward_quantized_on_oracle_operands(d, T):
     """The attention step alone, fed operands quantized by the oracle."""
