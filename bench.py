@@ -499,6 +499,27 @@ def run_gpu(args, rank, world, local_rank):
                  "uos_pnq_attn_speedup": nv_attn / attn_avg_ms, "kernel": f"mxattn_fwd_kernel<{w.d},{w.kv_tile},1,nvfp4>"}
         del wsn
 
+    # The ceiling of the attention kernel's own tensor-core instruction on this GPU:
+    # its M = N = 128, K = 64 block-scaled FP4 MMA issued back to back from shared
+    # memory, one CTA per SM (not part of the timed step).
+    mma_loop = None
+    if rank == 0 and not args.quick:
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        iters = 20000
+        mx.mxattn_mxf4_mma_loop(sms, iters, stream=stream)
+        torch.cuda.synchronize()
+        l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        l0.record(stream)
+        st = mx.mxattn_mxf4_mma_loop(sms, iters, stream=stream)
+        l1.record(stream)
+        torch.cuda.synchronize()
+        if int(st.item()) != 0:
+            raise RuntimeError("tensor-core loop reported a timeout")
+        loop_ms = l0.elapsed_time(l1)
+        mma_loop = {"tflops": sms * iters * mx.MXF4_LOOP_FLOP_PER_ITER / (loop_ms / 1e3) / 1e12, "ms": loop_ms,
+                    "ctas": sms, "iters": iters,
+                    "what": "tcgen05.mma kind::mxf4 block32, M=N=128, K=64, back to back from shared memory"}
+
     if rank == 0:
         attn_tflops = w.flops / (attn_avg_ms / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
@@ -521,7 +542,9 @@ def run_gpu(args, rank, world, local_rank):
                          "peak_source": f"{peak_kind} bf16 sustained {peaks['bf16_tflops_sustained']} TFLOP/s x "
                                         f"{FP4_PER_BF16:g} (nominal dense fp4:bf16)",
                          "attn_ms": attn_avg_ms, "prepare_ms": sum(prep_ms) / len(prep_ms),
-                         "frac_of_9pf_spec": attn_tflops / 9000.0},
+                         "frac_of_9pf_spec": attn_tflops / 9000.0,
+                         "mxf4_mma_loop": mma_loop,
+                         "frac_of_mxf4_mma_loop": None if mma_loop is None else attn_tflops / mma_loop["tflops"]},
             "cpu_baseline": base,
             "e2e": None if e2e_ms is None else {
                 "value": job_flops / (e2e_ms / 1e3) / 1e12, "unit": UNIT,

@@ -321,6 +321,23 @@ mxattn_status mxattn_nvfp4_attend(int B, int H, int N, int d, int kv_tile, int p
 mxattn_status mxattn_p_selftest(int path, const float* in, int64_t n, float qmax, int32_t* out,
                                 mxattn_stream_t stream);
 
+/*
+ * Measurement utility (this library's own; the paper has no counterpart): the
+ * throughput ceiling of the block-scaled FP4 tensor-core instruction the
+ * attention kernel uses.  Launches `ctas` CTAs; in each, one thread issues
+ * 2 * iters tcgen05.mma.kind::mxf4.block_scale.block32 instructions of shape
+ * M = 128, N = 128, K = 64 (the attention kernel's S = Q K^T shape and
+ * descriptors) back to back on operands held in shared memory, accumulating
+ * into one TMEM tile.  Work per launch: ctas * iters * 2 * (2 * 128 * 128 * 64)
+ * flop; time it with events on `stream`.
+ *   ctas in [1, 4096], iters in [1, 200000] (a launch then takes milliseconds);
+ *   status: device u32, 4-byte aligned; zeroed by the call, MXATTN_ERR_TIMEOUT
+ *     ORed in if the final wait gave up (2 s).
+ * Errors: MXATTN_ERR_INVALID (arguments), MXATTN_ERR_CUDA (launch failed).
+ * Asynchronous on `stream`.
+ */
+mxattn_status mxattn_mxf4_mma_loop(int ctas, int iters, uint32_t* status, mxattn_stream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* mxattn_status_string(mxattn_status status);
 

@@ -18,6 +18,7 @@ from .mxattn import (  # noqa: F401
     mxattn_nvfp4_forward,
     mxattn_nvfp4_prepare,
     mxattn_nvfp4_quantize,
+    mxattn_mxf4_mma_loop,
     mxattn_p_selftest,
     mxattn_prepare,
     mxattn_quantize,

@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.mxattn_wait_selftest.restype = i32
         L.mxattn_p_selftest.argtypes = [i32, P, i64, f32, P, P]
         L.mxattn_p_selftest.restype = i32
+        L.mxattn_mxf4_mma_loop.argtypes = [i32, i32, P, P]
+        L.mxattn_mxf4_mma_loop.restype = i32
         L.mxattn_nvfp4_quantize.argtypes = [P, i64, i64, P, P, P, P]
         L.mxattn_nvfp4_quantize.restype = i32
         L.mxattn_nvfp4_workspace_size.argtypes = [i32, i32, i32, i32]
@@ -91,7 +93,7 @@ def declared_symbols() -> list[str]:
     """Names of the entry points declared in include/mxattn.h."""
     with open(HEADER) as f:
         text = f.read()
-    return sorted(set(re.findall(r"\b(mxattn_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(mxattn_[a-z0-9_]+)\s*\(", text)))
 
 
 def status_string(status: int) -> str:
@@ -299,6 +301,20 @@ def mxattn_p_selftest(path: int, x: torch.Tensor, qmax: float = 7.25, out=None, 
     _check(lib().mxattn_p_selftest(int(path), _cuda(x, "x", torch.float32), x.numel(), float(qmax),
                                    _cuda(out, "out", torch.int32), _stream(stream)), "mxattn_p_selftest")
     return out
+
+
+MXF4_LOOP_FLOP_PER_ITER = 2 * (2 * 128 * 128 * 64)  # two K = 64 MMAs of M = N = 128 per iteration
+
+
+def mxattn_mxf4_mma_loop(ctas: int, iters: int, status=None, stream=None) -> torch.Tensor:
+    """Launch the tensor-core throughput loop (ctas CTAs, 2 * iters block-scaled
+    FP4 MMAs each, ctas * iters * MXF4_LOOP_FLOP_PER_ITER flop); returns the
+    device status word (0, or MXATTN_ERR_TIMEOUT once the stream has run it)."""
+    if status is None:
+        status = torch.empty(1, dtype=torch.int32, device=torch.device("cuda", torch.cuda.current_device()))
+    _check(lib().mxattn_mxf4_mma_loop(int(ctas), int(iters), _cuda(status, "status"), _stream(stream)),
+           "mxattn_mxf4_mma_loop")
+    return status
 
 
 def mxattn_status_string(status: int) -> str:

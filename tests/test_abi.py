@@ -19,7 +19,8 @@ def test_header_declares_the_boundary():
     syms = mx.declared_symbols()
     for name in ("mxattn_quantize", "mxattn_quantize_vt", "mxattn_workspace_size", "mxattn_forward",
                  "mxattn_forward_quantized", "mxattn_workspace_status", "mxattn_status_string", "mxattn_prepare",
-                 "mxattn_attend"):
+                 "mxattn_attend", "mxattn_nvfp4_forward", "mxattn_nvfp4_quantize", "mxattn_nvfp4_workspace_size",
+                 "mxattn_mxf4_mma_loop"):
         assert name in syms
 
 
@@ -143,6 +144,16 @@ def test_p_selftest_rejects_bad_arguments_before_launching(L):
     assert L.mxattn_p_selftest(0, None, 8, f(7.25), fake, None) == 1    # null input
     assert L.mxattn_p_selftest(0, _p((1 << 20) + 2), 8, f(7.25), fake, None) == 1  # misaligned
     assert L.mxattn_p_selftest(1, None, 0, f(7.25), None, None) == 0    # empty is a no-op
+
+
+def test_mma_loop_rejects_bad_arguments_before_launching(L):
+    fake = _p(1 << 20)
+    assert L.mxattn_mxf4_mma_loop(0, 10, fake, None) == 1          # no CTAs
+    assert L.mxattn_mxf4_mma_loop(5000, 10, fake, None) == 1       # too many CTAs
+    assert L.mxattn_mxf4_mma_loop(148, 0, fake, None) == 1         # no iterations
+    assert L.mxattn_mxf4_mma_loop(148, 200001, fake, None) == 1    # a launch would run too long
+    assert L.mxattn_mxf4_mma_loop(148, 10, None, None) == 1        # null status
+    assert L.mxattn_mxf4_mma_loop(148, 10, _p((1 << 20) + 2), None) == 1  # misaligned status
 
 
 def test_header_compiles_as_c_and_links(L, tmp_path):

@@ -1,0 +1,38 @@
+"""The tensor-core throughput loop (mxattn_mxf4_mma_loop): the block-scaled
+FP4 MMA shape of the attention kernel, issued back to back on shared-memory
+operands, finishes without a timeout, its time grows with the work, and its
+rate lies between the attention kernel's own rate on small launches and the
+nominal dense FP4 peak."""
+import pytest
+import torch
+
+from mxfp4_microscaled_quantization_b200 import mxattn as mx
+
+pytestmark = pytest.mark.gpu
+
+
+def _time(ctas, iters):
+    mx.mxattn_mxf4_mma_loop(ctas, iters)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    st = mx.mxattn_mxf4_mma_loop(ctas, iters)
+    e1.record()
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    return e0.elapsed_time(e1)
+
+
+def test_mma_loop_completes_and_scales():
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    t1 = _time(sms, 2000)
+    t2 = _time(sms, 8000)
+    assert 2.5 < t2 / t1 < 5.0, (t1, t2)
+    tflops = sms * 8000 * mx.MXF4_LOOP_FLOP_PER_ITER / (t2 / 1e3) / 1e12
+    print(f"[mxf4 loop] {sms} CTAs x 8000 iterations: {t2:.3f} ms, {tflops:.0f} TFLOP/s")
+    assert 1000 < tflops < 10000, tflops
+
+
+@pytest.mark.parametrize("ctas", [1, 7, 296])
+def test_mma_loop_other_grids(ctas):
+    assert _time(ctas, 500) > 0
