@@ -84,18 +84,63 @@ def profiled_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 100 ms during the timed region."""
+    """SM clock, its maximum and the clock-event (throttle) reasons of this
+    rank's GPU during the timed region: read every 10 ms by NVML in a
+    background thread (read only; the device is matched by PCI bus id), or
+    polled with nvidia-smi every 100 ms when NVML is unavailable."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.thread = None
+        self.samples = []  # (sm MHz, max sm MHz, reason names)
         self.path = os.path.join("/tmp", f"mxattn_clocks_{os.getpid()}.csv")
 
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+
+        pynvml.nvmlInit()
+        try:
+            pr = torch.cuda.get_device_properties(self.gpu)
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(
+                f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0".encode())
+        except Exception:  # noqa: BLE001 - older properties or bus-id formats: fall back to the index
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
     def __enter__(self):
+        import threading
+
+        try:
+            nv, h = self._nvml_handle()
+            smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            bits = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
+            self.stop = threading.Event()
+
+            def run():
+                while not self.stop.is_set():
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        mask = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    except Exception:  # noqa: BLE001 - a failed read is skipped, not fatal
+                        sm, mask = None, 0
+                    if sm is not None:
+                        self.samples.append((float(sm), float(smax), [n for n, bit in bits if mask & bit]))
+                    self.stop.wait(0.01)
+
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:  # noqa: BLE001 - no NVML: poll nvidia-smi instead
+            self.thread = None
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -106,6 +151,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -115,27 +163,29 @@ class ClockSampler:
             self.fh.close()
 
     def summary(self):
-        if self.proc is None:
-            return None
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        try:
-            os.remove(self.path)
-        except OSError:
-            pass
+        source = "nvml"
+        rows = list(self.samples)
+        if self.thread is None:
+            if self.proc is None:
+                return None
+            source = "nvidia-smi"
+            names = [n for n, _ in self.REASONS]
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9 and parts[1].replace(".", "").isdigit() and parts[2].replace(".", "").isdigit():
+                        rows.append((float(parts[1]), float(parts[2]),
+                                     [names[i] for i in range(4) if parts[5 + i].lower().startswith("active")]))
+            try:
+                os.remove(self.path)
+            except OSError:
+                pass
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
-        loaded = [s for s in sm if smax and s >= 0.3 * max(smax)] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons, "samples": len(rows)}
+        smax = max(r[1] for r in rows)
+        loaded = [r[0] for r in rows if r[0] >= 0.3 * smax] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
+                "reasons": sorted({n for r in rows for n in r[2]}), "samples": len(rows), "source": source}
 
 
 def oracle_sample(Q, K, V, w, rows, nthreads=0):
