@@ -21,7 +21,7 @@
  *     and K; the online softmax walks key tiles of kv_tile columns in
  *     ascending order and subtracts the running maximum after each tile.
  *   - PNQ off: P*V still uses the quantized exponentials but the row sum uses
- *     the unquantized ones (the abstract's "row-wise normalization error").
+ *     the unquantized ones (the error in the row-wise normalization that the abstract names).
  *
  * Conventions for every entry point:
  *   - Pointers are device pointers unless stated otherwise; the caller owns
@@ -60,7 +60,7 @@ typedef enum {
 
 typedef enum {
     MXATTN_RULE_OCP = 0, /* e = floor(log2 amax) - 2 */
-    MXATTN_RULE_UOS = 1  /* smallest e with amax <= 7.25 * 2^e (abstract: "Qmax=7.25") */
+    MXATTN_RULE_UOS = 1  /* smallest e with amax <= 7.25 * 2^e (the abstract's Qmax) */
 } mxattn_rule;
 
 /*
@@ -75,7 +75,7 @@ typedef enum {
  */
 
 /*
- * Standalone MXFP4 quantize/pack (the abstract's "direct MXFP4 quantization";
+ * Standalone MXFP4 quantize/pack (the abstract's direct MXFP4 quantization;
  * the scale rule is UOS or OCP).
  *   x:      bf16 [rows, cols], cols % 32 == 0, 16-byte aligned.
  *   codes:  u8 [rows, cols/2] (packed E2M1), 4-byte aligned.
@@ -233,7 +233,7 @@ mxattn_status mxattn_wait_selftest(int arrive, unsigned timeout_us, unsigned* ou
 
 /* ---------------------------------------------------------------------------
  * NVFP4 comparison variant.  The abstract measures MXAttention against
- * "NVFP4-based baselines" without defining them; this library's reading is
+ * NVFP4 baselines without defining them; this library's reading is
  * NVIDIA's NVFP4 applied to the same four operands and the same softmax loop:
  *   - E2M1 elements (as above) in blocks of 16 along the contraction axis,
  *     one unsigned E4M3 (OCP FP8 E4M3) scale per block, and one fp32

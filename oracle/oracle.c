@@ -42,7 +42,7 @@
 /* E2M1 magnitudes in code order (code bits: sign | exponent(2) | mantissa(1)). */
 static const double kE2M1Magnitude[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
 
-/* UOS boundary, from the abstract: "optimal scaling boundary Qmax=7.25". */
+/* UOS boundary: the abstract fixes the optimal scale boundary at Qmax = 7.25. */
 static const double kUosQmax = 7.25;
 
 /* bfloat16 bit pattern -> value: the top 16 bits of an IEEE binary32. */
@@ -219,10 +219,10 @@ void oracle_dequantize_rows(const uint8_t* codes, const uint8_t* scales, int64_t
  * pnq = 1: PNQ (abstract: quantize the unnormalized exponentials before the
  * row-wise summation, so the row sum is built from the same quantized values
  * that weight V).  pnq = 0: the row sum uses the unquantized exponentials
- * while P*V uses the quantized ones -- the "row-wise normalization error" the
+ * while P*V uses the quantized ones -- the error in the row-wise normalization that the
  * abstract attributes to plain MXFP4 attention (reading).
  *
- * The softmax loop (abstract: "the softmax loop"; reading: the standard
+ * The softmax loop (the abstract's softmax loop; reading: the standard
  * online softmax over key tiles of kv_tile columns, ascending), per row i:
  *   s_j   = (deq(Q_i) . deq(K_j)) * scale      (scale applied after quantization: reading)
  *   m = -inf, l = 0, o = 0
@@ -368,7 +368,7 @@ int oracle_max_threads(void) {
 /* ======================================================================
  * NVFP4 comparison variant.
  *
- * The abstract compares MXAttention with "strong NVFP4-based baselines" and
+ * The abstract compares MXAttention with NVFP4 baselines and
  * gives no definition of them.  Reading: NVIDIA's NVFP4 format -- E2M1
  * elements in blocks of 16 with one unsigned E4M3 (OCP FP8 E4M3) scale per
  * block, and a second, per-tensor fp32 scale -- applied to the same four

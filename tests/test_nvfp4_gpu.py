@@ -1,4 +1,4 @@
-"""Parity of the NVFP4 comparison variant (the "NVFP4-based baselines" of the
+"""Parity of the NVFP4 comparison variant (the NVFP4 baselines of the
 MXAttention abstract, "MXAttention: Data-Free Optimal Scaling and
 Pre-Normalization Quantization for MXFP4 Attention") with the CPU oracle.
 

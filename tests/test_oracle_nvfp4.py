@@ -1,6 +1,6 @@
 """Pins of the oracle's NVFP4 comparison variant (CPU).
 
-The MXAttention abstract compares against "NVFP4-based baselines" without
+The MXAttention abstract compares against NVFP4 baselines without
 defining them; the oracle's reading (oracle.c, "NVFP4 comparison variant") is
 NVIDIA's NVFP4: E2M1 elements in blocks of 16, one E4M3 scale per block and a
 per-(batch, head) fp32 scale g = 448 / amax, scale arithmetic in fp32.  The
