@@ -333,10 +333,15 @@ mxattn_status mxattn_p_selftest(int path, const float* in, int64_t n, float qmax
  *   ctas in [1, 4096], iters in [1, 200000] (a launch then takes milliseconds);
  *   status: device u32, 4-byte aligned; zeroed by the call, MXATTN_ERR_TIMEOUT
  *     ORed in if the final wait gave up (2 s).
+ *   cycles: device u64 [ctas], 8-byte aligned, or NULL; CTA i writes the SM
+ *     clock cycles from its first issue to the completion of its last MMA, so
+ *     the rate per clock (2 * iters * 2 * 128 * 128 * 64 / cycles per SM, with
+ *     one CTA per SM) does not depend on the clock the power cap allows.
  * Errors: MXATTN_ERR_INVALID (arguments), MXATTN_ERR_CUDA (launch failed).
  * Asynchronous on `stream`.
  */
-mxattn_status mxattn_mxf4_mma_loop(int ctas, int iters, uint32_t* status, mxattn_stream_t stream);
+mxattn_status mxattn_mxf4_mma_loop(int ctas, int iters, uint32_t* status, uint64_t* cycles,
+                                   mxattn_stream_t stream);
 
 /* Static, NUL-terminated description of a status code. */
 const char* mxattn_status_string(mxattn_status status);

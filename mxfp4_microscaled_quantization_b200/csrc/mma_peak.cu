@@ -9,7 +9,9 @@
 // operands that stay in shared memory, so nothing but the tensor core is
 // timed.  The operands are a fixed mix of E2M1 codes with unit scales; the
 // result is never read.  The one wait (for the final commit) is bounded like
-// every wait in the library.
+// every wait in the library.  Each CTA also records the SM clock cycles from
+// its first issue to the completion of its last MMA, so the rate can be
+// stated per clock, independent of the clock the power cap allows.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -32,7 +34,8 @@ __device__ __forceinline__ uint64_t atom_desc(const void* p) {
     return smem_desc(smem_u32(p), 0, 128, kLayoutNone);
 }
 
-__global__ void __launch_bounds__(kThreads) mxf4_mma_loop_kernel(int iters, uint32_t* status) {
+__global__ void __launch_bounds__(kThreads) mxf4_mma_loop_kernel(int iters, uint32_t* status,
+                                                                  unsigned long long* cycles) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;           // 128 rows x 64 bytes (K = 128 E2M1 values), 64-byte swizzle
@@ -61,7 +64,10 @@ __global__ void __launch_bounds__(kThreads) mxf4_mma_loop_kernel(int iters, uint
     tc_fence_after_sync();
     const uint32_t tbase = tmem_holder;
     if (warp == 0) {
-        if (elect_one_sync()) {
+        const bool leader = elect_one_sync();
+        unsigned long long t0 = 0;
+        if (leader) {
+            t0 = clock64();
             tc_cp_sf(tbase + 128, atom_desc(sSf));
             tc_cp_sf(tbase + 132, atom_desc(sSf + 512));
             const uint64_t adesc = smem_desc(smem_u32(sA), 16, 512, kLayoutSw64);
@@ -76,6 +82,7 @@ __global__ void __launch_bounds__(kThreads) mxf4_mma_loop_kernel(int iters, uint
         }
         __syncwarp();
         mbar_wait_bounded(&bar, 0, &abort_flag, status, kTimeoutCode, kLoopTimeoutNs);
+        if (leader && cycles != nullptr) cycles[blockIdx.x] = clock64() - t0;
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -88,12 +95,14 @@ __global__ void __launch_bounds__(kThreads) mxf4_mma_loop_kernel(int iters, uint
 }  // namespace
 }  // namespace mxattn
 
-MXATTN_API mxattn_status mxattn_mxf4_mma_loop(int ctas, int iters, uint32_t* status, mxattn_stream_t stream) {
+MXATTN_API mxattn_status mxattn_mxf4_mma_loop(int ctas, int iters, uint32_t* status, uint64_t* cycles,
+                                              mxattn_stream_t stream) {
     if (ctas < 1 || ctas > 4096 || iters < 1 || iters > 200000 || status == nullptr ||
-        (reinterpret_cast<uintptr_t>(status) & 3u))
+        (reinterpret_cast<uintptr_t>(status) & 3u) || (reinterpret_cast<uintptr_t>(cycles) & 7u))
         return MXATTN_ERR_INVALID;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(status, 0, sizeof(uint32_t), s) != cudaSuccess) return MXATTN_ERR_CUDA;
-    mxattn::mxf4_mma_loop_kernel<<<ctas, mxattn::kThreads, mxattn::kSmemBytes, s>>>(iters, status);
+    mxattn::mxf4_mma_loop_kernel<<<ctas, mxattn::kThreads, mxattn::kSmemBytes, s>>>(
+        iters, status, reinterpret_cast<unsigned long long*>(cycles));
     return cudaGetLastError() == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
 }

@@ -73,7 +73,7 @@ def lib() -> ctypes.CDLL:
         L.mxattn_wait_selftest.restype = i32
         L.mxattn_p_selftest.argtypes = [i32, P, i64, f32, P, P]
         L.mxattn_p_selftest.restype = i32
-        L.mxattn_mxf4_mma_loop.argtypes = [i32, i32, P, P]
+        L.mxattn_mxf4_mma_loop.argtypes = [i32, i32, P, P, P]
         L.mxattn_mxf4_mma_loop.restype = i32
         L.mxattn_nvfp4_quantize.argtypes = [P, i64, i64, P, P, P, P]
         L.mxattn_nvfp4_quantize.restype = i32
@@ -306,13 +306,21 @@ def mxattn_p_selftest(path: int, x: torch.Tensor, qmax: float = 7.25, out=None, 
 MXF4_LOOP_FLOP_PER_ITER = 2 * (2 * 128 * 128 * 64)  # two K = 64 MMAs of M = N = 128 per iteration
 
 
-def mxattn_mxf4_mma_loop(ctas: int, iters: int, status=None, stream=None) -> torch.Tensor:
+def mxattn_mxf4_mma_loop(ctas: int, iters: int, status=None, cycles=None, stream=None) -> torch.Tensor:
     """Launch the tensor-core throughput loop (ctas CTAs, 2 * iters block-scaled
     FP4 MMAs each, ctas * iters * MXF4_LOOP_FLOP_PER_ITER flop); returns the
-    device status word (0, or MXATTN_ERR_TIMEOUT once the stream has run it)."""
+    device status word (0, or MXATTN_ERR_TIMEOUT once the stream has run it).
+    `cycles`: optional device int64 [ctas] that receives each CTA's SM clock
+    cycles from first issue to last completion."""
+    dev = torch.device("cuda", torch.cuda.current_device())
     if status is None:
-        status = torch.empty(1, dtype=torch.int32, device=torch.device("cuda", torch.cuda.current_device()))
-    _check(lib().mxattn_mxf4_mma_loop(int(ctas), int(iters), _cuda(status, "status"), _stream(stream)),
+        status = torch.empty(1, dtype=torch.int32, device=dev)
+    cyc = None
+    if cycles is not None:
+        if cycles.dtype != torch.int64 or cycles.numel() < ctas or not cycles.is_cuda:
+            raise MxattnError(1, "cycles must be a CUDA int64 tensor with at least `ctas` elements")
+        cyc = _cuda(cycles, "cycles")
+    _check(lib().mxattn_mxf4_mma_loop(int(ctas), int(iters), _cuda(status, "status"), cyc, _stream(stream)),
            "mxattn_mxf4_mma_loop")
     return status
 

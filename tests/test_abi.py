@@ -148,12 +148,13 @@ def test_p_selftest_rejects_bad_arguments_before_launching(L):
 
 def test_mma_loop_rejects_bad_arguments_before_launching(L):
     fake = _p(1 << 20)
-    assert L.mxattn_mxf4_mma_loop(0, 10, fake, None) == 1          # no CTAs
-    assert L.mxattn_mxf4_mma_loop(5000, 10, fake, None) == 1       # too many CTAs
-    assert L.mxattn_mxf4_mma_loop(148, 0, fake, None) == 1         # no iterations
-    assert L.mxattn_mxf4_mma_loop(148, 200001, fake, None) == 1    # a launch would run too long
-    assert L.mxattn_mxf4_mma_loop(148, 10, None, None) == 1        # null status
-    assert L.mxattn_mxf4_mma_loop(148, 10, _p((1 << 20) + 2), None) == 1  # misaligned status
+    assert L.mxattn_mxf4_mma_loop(0, 10, fake, None, None) == 1          # no CTAs
+    assert L.mxattn_mxf4_mma_loop(5000, 10, fake, None, None) == 1       # too many CTAs
+    assert L.mxattn_mxf4_mma_loop(148, 0, fake, None, None) == 1         # no iterations
+    assert L.mxattn_mxf4_mma_loop(148, 200001, fake, None, None) == 1    # a launch would run too long
+    assert L.mxattn_mxf4_mma_loop(148, 10, None, None, None) == 1        # null status
+    assert L.mxattn_mxf4_mma_loop(148, 10, _p((1 << 20) + 2), None, None) == 1  # misaligned status
+    assert L.mxattn_mxf4_mma_loop(148, 10, fake, _p((1 << 20) + 4), None) == 1  # misaligned cycles
 
 
 def test_header_compiles_as_c_and_links(L, tmp_path):
