@@ -51,41 +51,46 @@ def lib():
     global _lib
     if _lib is None:
         build()
-        L = ctypes.CDLL(_LIB_PATH)
-        P = ctypes.c_void_p
-        i64 = ctypes.c_int64
-        L.oracle_e2m1_encode_batch.argtypes = [P, i64, P]
-        L.oracle_scale_exponent_batch.argtypes = [P, i64, ctypes.c_int, P]
-        L.oracle_scale_exponent_q_batch.argtypes = [P, i64, ctypes.c_int, ctypes.c_double, P]
-        L.oracle_quantize_rows_q.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_double, P, P]
-        L.oracle_quantize_cols_q.argtypes = [P, i64, i64, i64, ctypes.c_int, ctypes.c_double, P, P]
-        L.oracle_attention_head_q.argtypes = [P, P, P, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_double,
-                                              ctypes.c_int, ctypes.c_double, P, i64, P, ctypes.c_int]
-        L.oracle_attention_head_q.restype = ctypes.c_int
-        L.oracle_quantize_rows.argtypes = [P, i64, i64, ctypes.c_int, P, P]
-        L.oracle_quantize_cols.argtypes = [P, i64, i64, i64, ctypes.c_int, P, P]
-        L.oracle_dequantize_rows.argtypes = [P, P, i64, i64, P]
-        L.oracle_attention_head.argtypes = [P, P, P, i64, i64, i64, ctypes.c_int, ctypes.c_int,
-                                            ctypes.c_int, ctypes.c_double, P, i64, P, ctypes.c_int]
-        L.oracle_attention_head.restype = ctypes.c_int
-        L.oracle_max_threads.restype = ctypes.c_int
-        L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
-        L.oracle_e2m1_decode.restype = ctypes.c_double
-        L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
-        L.oracle_e4m3_decode.restype = ctypes.c_double
-        L.oracle_e4m3_encode_batch.argtypes = [P, i64, P]
-        L.oracle_nvfp4_global.argtypes = [ctypes.c_double]
-        L.oracle_nvfp4_global.restype = ctypes.c_float
-        L.oracle_bf16_amax.argtypes = [P, i64]
-        L.oracle_bf16_amax.restype = ctypes.c_double
-        L.oracle_nvfp4_quantize_rows.argtypes = [P, i64, i64, ctypes.c_float, P, P]
-        L.oracle_nvfp4_quantize_cols.argtypes = [P, i64, i64, i64, P, P, P]
-        L.oracle_nvfp4_dequantize_rows.argtypes = [P, P, i64, i64, ctypes.c_float, P]
-        L.oracle_nvfp4_attention_head.argtypes = [P, P, P, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                                  ctypes.c_double, P, i64, P, ctypes.c_int]
-        L.oracle_nvfp4_attention_head.restype = ctypes.c_int
-        _lib = L
+        _lib = load(_LIB_PATH)
     return _lib
+
+
+def load(path: str) -> ctypes.CDLL:
+    """Open a compiled oracle library at `path` and declare its signatures."""
+    L = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    i64 = ctypes.c_int64
+    L.oracle_e2m1_encode_batch.argtypes = [P, i64, P]
+    L.oracle_scale_exponent_batch.argtypes = [P, i64, ctypes.c_int, P]
+    L.oracle_scale_exponent_q_batch.argtypes = [P, i64, ctypes.c_int, ctypes.c_double, P]
+    L.oracle_quantize_rows_q.argtypes = [P, i64, i64, ctypes.c_int, ctypes.c_double, P, P]
+    L.oracle_quantize_cols_q.argtypes = [P, i64, i64, i64, ctypes.c_int, ctypes.c_double, P, P]
+    L.oracle_attention_head_q.argtypes = [P, P, P, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                          ctypes.c_int, ctypes.c_double, P, i64, P, ctypes.c_int]
+    L.oracle_attention_head_q.restype = ctypes.c_int
+    L.oracle_quantize_rows.argtypes = [P, i64, i64, ctypes.c_int, P, P]
+    L.oracle_quantize_cols.argtypes = [P, i64, i64, i64, ctypes.c_int, P, P]
+    L.oracle_dequantize_rows.argtypes = [P, P, i64, i64, P]
+    L.oracle_attention_head.argtypes = [P, P, P, i64, i64, i64, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_int, ctypes.c_double, P, i64, P, ctypes.c_int]
+    L.oracle_attention_head.restype = ctypes.c_int
+    L.oracle_max_threads.restype = ctypes.c_int
+    L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+    L.oracle_e2m1_decode.restype = ctypes.c_double
+    L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    L.oracle_e4m3_decode.restype = ctypes.c_double
+    L.oracle_e4m3_encode_batch.argtypes = [P, i64, P]
+    L.oracle_nvfp4_global.argtypes = [ctypes.c_double]
+    L.oracle_nvfp4_global.restype = ctypes.c_float
+    L.oracle_bf16_amax.argtypes = [P, i64]
+    L.oracle_bf16_amax.restype = ctypes.c_double
+    L.oracle_nvfp4_quantize_rows.argtypes = [P, i64, i64, ctypes.c_float, P, P]
+    L.oracle_nvfp4_quantize_cols.argtypes = [P, i64, i64, i64, P, P, P]
+    L.oracle_nvfp4_dequantize_rows.argtypes = [P, P, i64, i64, ctypes.c_float, P]
+    L.oracle_nvfp4_attention_head.argtypes = [P, P, P, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_double, P, i64, P, ctypes.c_int]
+    L.oracle_nvfp4_attention_head.restype = ctypes.c_int
+    return L
 
 
 def _ptr(a: np.ndarray):
