@@ -44,12 +44,21 @@ ATTN_SOURCES = tuple(os.path.join(ROOT, "mxfp4_microscaled_quantization_b200", "
                      for f in ("attention.cu", "ptx.cuh"))
 
 
-def config_dict(w=WORKLOAD):
+PARALLELISM = {
+    "heads": "heads sharded over {world} ranks (one problem, no exchange)",
+    "sequence": "tokens sharded over {world} ranks (one problem; all-to-all to heads and back, NCCL)",
+    "replicas": "{world} independent replicas (one batch per rank)"}
+
+
+def config_dict(w=WORKLOAD, world=1, shard="replicas"):
+    """The workload the line is quoted on; both arms (ours and the reference) print the same dict."""
+    gb = 3 * w.B * w.H * w.N * w.d * 2 / 1e9
     return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} ({w.frames}x{w.rows}x{w.cols} tokens) d={w.d} "
                         f"kv_tile={w.kv_tile}, UOS + PNQ, smooth low-rank + noise bf16 inputs",
             "B": w.B, "H": w.H, "N": w.N, "d": w.d, "kv_tile": w.kv_tile, "rule": "uos", "pnq": True,
             "step": "mxattn_prepare (Q/K + V^T quantize) + mxattn_attend (fused attention)",
-            "l2": "inputs larger than L2: 1.0 GB of bf16 Q/K/V per step (no flush)"}
+            "l2": f"inputs larger than L2: {gb:.1f} GB of bf16 Q/K/V per step (no flush)",
+            "parallelism": PARALLELISM[shard].format(world=world)}
 
 
 def load_peaks():
@@ -232,7 +241,7 @@ def run_reference(args, rank, world):
     Q, K, V = wl.make_qkv(w, seed=0)
     threads = oracle.max_threads()
     # size one step to a bounded sample so warmup + steps stay within a few minutes
-    step_budget_s = max(2.0, 120.0 / (args.warmup + args.steps))
+    step_budget_s = args.ref_step_budget or max(2.0, 120.0 / (args.warmup + args.steps))
     rows0, _ = sized_oracle_rows(Q, K, V, w, step_budget_s, threads)
     n = len(rows0)
     times = []
@@ -247,7 +256,7 @@ def run_reference(args, rank, world):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": config_dict(),
+            "config": config_dict(w, world, args.shard),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": f"per step {n} seeded query rows of head 0 (with that head's K/V "
                                        f"quantization) on {threads} OpenMP threads"},
@@ -256,31 +265,78 @@ def run_reference(args, rank, world):
     return 0
 
 
-def quantize_sweep_point(torch, mx, peaks, peak_kind, log2n=30, iters=10):
-    """Standalone quantize kernel on the largest quantize-sweep size (2^30 bf16 elements)."""
-    x = wl.student_t_matrix(1 << log2n, 4096, seed=0)
+QUANT_SWEEP_LOG2 = (20, 24, 27, 30)
+
+
+def quantize_sweep(torch, mx, peaks, peak_kind, iters=10):
+    """The standalone quantize kernel (mxattn_quantize) on the config-5 sweep:
+    0.5 * StudentT(3) bf16 [2^k / 4096, 4096] for k in 20, 24, 27, 30 (the first
+    2^k elements of one seeded 2^30-element draw), OCP and UOS.  Every launch is
+    timed on its own with CUDA events, after a 512 MB write that flushes L2
+    (the smaller sizes fit in L2); GB/s counts 2.53125 bytes per element."""
+    big = max(QUANT_SWEEP_LOG2)
+    x = wl.student_t_matrix(1 << big, 4096, seed=0)
     xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
     del x
     codes = torch.empty((xd.shape[0], 2048), dtype=torch.uint8, device="cuda")
     scales = torch.empty((xd.shape[0], 128), dtype=torch.uint8, device="cuda")
-    for _ in range(3):
-        mx.mxattn_quantize(xd, "uos", codes, scales)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(iters):
-        mx.mxattn_quantize(xd, "uos", codes, scales)
-    e1.record()
-    torch.cuda.synchronize()
-    t = e0.elapsed_time(e1) / 1e3 / iters
-    nbytes = (1 << log2n) * (2 + 0.5 + 1 / 32)
-    gbs = nbytes / t / 1e9
-    out = {"elements": 1 << log2n, "bytes_per_element": 2.53125, "us_per_launch": t * 1e6, "achieved_gbs": gbs,
-           "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
-           "frac_of_8tbs_spec": gbs / 8000.0, "peak_kind": peak_kind, "rule": "uos"}
-    del xd, codes, scales
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    points = []
+    for k in QUANT_SWEEP_LOG2:
+        rows = (1 << k) // 4096
+        xs, cs, ss = xd[:rows], codes[:rows], scales[:rows]
+        for rule in ("ocp", "uos"):
+            for _ in range(3):
+                mx.mxattn_quantize(xs, rule, cs, ss)
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+            for e0, e1 in ev:
+                flush.fill_(k & 0xFF)
+                e0.record()
+                mx.mxattn_quantize(xs, rule, cs, ss)
+                e1.record()
+            torch.cuda.synchronize()
+            t = sum(e0.elapsed_time(e1) for e0, e1 in ev) / iters / 1e3
+            gbs = (1 << k) * 2.53125 / t / 1e9
+            points.append({"log2_elements": k, "rule": rule, "us_per_launch": t * 1e6, "achieved_gbs": gbs,
+                           "frac": gbs / peaks["hbm_gbs"], "frac_of_8tbs_spec": gbs / 8000.0})
+    del xd, codes, scales, flush
     torch.cuda.empty_cache()
-    return out
+    return {"points": points, "bytes_per_element": 2.53125, "peak_gbs": peaks["hbm_gbs"], "peak_kind": peak_kind,
+            "shape": "[2^k / 4096, 4096] bf16, 0.5 * StudentT(3), seed 0", "l2": "512 MB written before every launch"}
+
+
+def long_video_leg(torch, mx, steps=3):
+    """The long video-DiT workload (B=1, H=24, N=75600, d=128, kv_tile=128, UOS +
+    PNQ): the same step (prepare + attend), attention and step times from CUDA
+    events, inputs generated by the same recipe (seed 0)."""
+    w = wl.WORKLOADS["long_video_dit"]
+    Q, K, V = wl.make_qkv(w, seed=0)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)  # noqa: E731
+    q, k, v = to_dev(Q), to_dev(K), to_dev(V)
+    del Q, K, V
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device="cuda")
+    ws = mx.new_workspace(w.B, w.H, w.N, w.d)
+    for _ in range(2):
+        mx.mxattn_prepare(q, k, v, "uos", ws)
+        mx.mxattn_attend(ws, w.B, w.H, w.N, w.d, w.kv_tile, True, "uos", 0.0, out)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for e in ev:
+        e[0].record()
+        mx.mxattn_prepare(q, k, v, "uos", ws)
+        e[1].record()
+        mx.mxattn_attend(ws, w.B, w.H, w.N, w.d, w.kv_tile, True, "uos", 0.0, out)
+        e[2].record()
+    torch.cuda.synchronize()
+    if mx.mxattn_workspace_status(ws) != 0:
+        raise RuntimeError("attention kernel reported a timeout (long video-DiT)")
+    attn = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+    step = sum(e[0].elapsed_time(e[2]) for e in ev) / steps
+    del q, k, v, out, ws
+    torch.cuda.empty_cache()
+    return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} kv_tile={w.kv_tile}, UOS + PNQ",
+            "attn_ms": attn, "step_ms": step, "attn_tflops": w.flops / (attn / 1e3) / 1e12,
+            "step_tflops": w.flops / (step / 1e3) / 1e12, "steps": steps}
 
 
 # MUFU exponentials per S element in mxattn_fwd_kernel with PNQ: 8 of every 16
@@ -494,7 +550,10 @@ def run_gpu(args, rank, world, local_rank):
 
     quant = None
     if rank == 0 and not args.quick and not args.no_quantize_sweep and not seq:
-        quant = quantize_sweep_point(torch, mx, peaks, peak_kind)
+        quant = quantize_sweep(torch, mx, peaks, peak_kind)
+    long_leg = None
+    if rank == 0 and not args.quick and not seq and args.workload == "video_dit" and not args.heads:
+        long_leg = long_video_leg(torch, mx)
 
     # The same attention step under every scale rule x PNQ combination: OCP
     # without PNQ is the comparator the method is measured against; the two mixed
@@ -577,7 +636,9 @@ def run_gpu(args, rank, world, local_rank):
 
     if rank == 0:
         attn_tflops = w.flops / (attn_avg_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
+        # Each launch is timed on its own, inside a sub-second region, and holds the maximum
+        # SM clock (see `clocks`): the burst bf16 figure is the matching denominator.
+        peak = peaks["bf16_tflops"] * FP4_PER_BF16
         clocks = clk.summary()
         mxf4_frac = None
         if mma_loop is not None:
@@ -591,16 +652,13 @@ def run_gpu(args, rank, world, local_rank):
             "scaling": "strong" if args.shard in ("heads", "sequence") else "weak",
             "vs_baseline": None, "data": "synthetic",
             "dtype": ("nvfp4 (e2m1 x e4m3, fp32 accumulate)" if nv_step else "mxfp4 (e2m1 x e8m0, fp32 accumulate)"),
-            "config": {**config_dict(w_full), "parallelism": {
-                "heads": f"heads sharded over {world} ranks (one problem, no exchange)",
-                "sequence": f"tokens sharded over {world} ranks (one problem; all-to-all to heads and back, NCCL)",
-                "replicas": f"{world} independent replicas (one batch per rank)"}[args.shard]},
+            "config": config_dict(w_full, world, args.shard),
             "pct_of_fp4_peak": 100.0 * value / world / peak,
             "roofline": {"bound": "tensor", "achieved": attn_tflops,
                          "kernel": f"mxattn_fwd_kernel<{w.d},{w.kv_tile}{',nvfp4' if nv_step else ''}>",
                          "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
                          "traffic": profiled_traffic() if (w == WORKLOAD and not nv_step) else None,
-                         "peak_source": f"{peak_kind} bf16 sustained {peaks['bf16_tflops_sustained']} TFLOP/s x "
+                         "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
                                         f"{FP4_PER_BF16:g} (nominal dense fp4:bf16)",
                          "attn_ms": attn_avg_ms, "prepare_ms": sum(prep_ms) / len(prep_ms),
                          "frac_of_9pf_spec": attn_tflops / 9000.0,
@@ -610,7 +668,8 @@ def run_gpu(args, rank, world, local_rank):
             "e2e": None if e2e_ms is None else {
                 "value": job_flops / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": 3 * B * H * N * d * 2, "d2h_bytes_per_step": B * H * N * d * 4,
-                "ms_per_step": e2e_ms, "api": "attention_from_host -> mxattn_forward",
+                "ms_per_step": e2e_ms, "steps": args.steps,
+                "api": "mxattn_forward_host (C ABI, pinned host buffers)",
                 "pipeline": "16 groups of (batch, head) slices; H2D, attention and D2H overlap on three streams"},
             "mufu_roofline": mufu_roofline(w, attn_avg_ms, clocks),
             "uos_pnq_overhead": overhead,
@@ -618,6 +677,7 @@ def run_gpu(args, rank, world, local_rank):
             "gpu_launches": (4 if nv_step else 3) * args.steps,
             "clocks": clocks,
             "quantize_sweep": quant,
+            "long_video_dit": long_leg,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -637,7 +697,7 @@ def measure_e2e(torch, mx, Q, K, V, w, bufs, stream, args, dist):
     for _ in range(2):
         mx.attention_from_host(q_h, k_h, v_h, w.kv_tile, True, "uos", 0.0, bufs, o_h)
     torch.cuda.synchronize()
-    e2e_steps = max(2, min(args.steps, 5))
+    e2e_steps = args.steps
     if dist is not None:
         dist.barrier()
     ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -647,6 +707,19 @@ def measure_e2e(torch, mx, Q, K, V, w, bufs, stream, args, dist):
     ee1.record(stream)
     torch.cuda.synchronize()
     return max_over_ranks([ee0.elapsed_time(ee1) / e2e_steps], dist, "cuda")[0]
+
+
+def launch_ranks(n: int) -> int:
+    """`--gpus N` outside torchrun: start N ranks of this same command on this node
+    (torch.distributed.run, rendezvous on 127.0.0.1); rank 0 prints the line."""
+    import socket
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
 
 
 def main():
@@ -670,7 +743,11 @@ def main():
                     help="instead of the timed step: O error against exact attention over scale boundaries in [6, 8]")
     ap.add_argument("--quick", action="store_true",
                     help="timed steps only: no CPU baseline, no end-to-end leg, no quantize sweep")
+    ap.add_argument("--ref-step-budget", type=float, default=0.0,
+                    help="--impl reference: seconds of oracle work per step (default: about 2 minutes in all)")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return launch_ranks(args.gpus)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

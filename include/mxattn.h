@@ -178,6 +178,45 @@ mxattn_status mxattn_forward_quantized(const uint8_t* q_codes, const uint8_t* q_
                                        mxattn_stream_t stream);
 
 /*
+ * mxattn_forward from host buffers to host buffers, with the transfers
+ * overlapped against the attention (a deployment entry point; the paper has
+ * no counterpart).  The (batch, head) slices are independent, so they are
+ * processed in groups: the copy to the device of group i+1 (one
+ * cudaMemcpyAsync each for Q, K, V) and the copy back of group i-1 overlap
+ * the attention of group i (one mxattn_forward per group on `stream`).
+ *   Q, K, V:   HOST bf16 [B, H, N, d]; O: HOST fp32 [B, H, N, d].  Page-locked
+ *              (pinned) host memory lets the copies run asynchronously; with
+ *              pageable memory the call still works but the copies do not
+ *              overlap.
+ *   q_dev, k_dev, v_dev: device bf16 [B, H, N, d] staging buffers, o_dev:
+ *              device fp32 [B, H, N, d], each 16-byte aligned.
+ *   workspace: device, 256-byte aligned, at least
+ *              mxattn_forward_host_workspace_size(B, H, N, d, group_sizes,
+ *              ngroups) bytes (the workspace of the largest group); its
+ *              status word holds the last group's timeout status
+ *              (mxattn_workspace_status).
+ *   group_sizes: NULL, or ngroups positive group sizes (in slices) that sum
+ *              to B*H, processed in order.  With NULL, ngroups groups
+ *              (0: 16; at most B*H): the first and the last of one slice each
+ *              (the only transfers nothing overlaps), the rest as equal as
+ *              possible.
+ * The copies run on two streams the call creates (one per direction); events
+ * order them against `stream`, which waits for the last copy back: when
+ * `stream` reaches the point after this call, O holds the result.  The
+ * streams and events are released by the runtime once that work is done.
+ * Argument errors as mxattn_forward, plus MXATTN_ERR_INVALID for a null or
+ * misaligned buffer, bad group sizes or a small workspace; MXATTN_ERR_CUDA if
+ * a stream, event or copy call fails (work already enqueued stays ordered
+ * before later work on `stream`).
+ */
+size_t mxattn_forward_host_workspace_size(int B, int H, int N, int d, const int* group_sizes, int ngroups);
+mxattn_status mxattn_forward_host(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                  int kv_tile, int pnq, mxattn_rule rule, float softmax_scale, float* O,
+                                  void* q_dev, void* k_dev, void* v_dev, float* o_dev, void* workspace,
+                                  size_t workspace_bytes, const int* group_sizes, int ngroups,
+                                  mxattn_stream_t stream);
+
+/*
  * mxattn_forward without a caller-provided workspace, for callers that cannot
  * allocate device memory themselves: code embedded in a host framework that
  * owns all device memory through its own pool and forbids raw cudaMalloc, or

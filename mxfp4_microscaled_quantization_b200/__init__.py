@@ -10,6 +10,8 @@ from .mxattn import (  # noqa: F401
     MxattnError,
     attention_from_host,
     declared_symbols,
+    forward_host_workspace_size,
+    host_groups,
     mxattn_attend,
     mxattn_forward,
     mxattn_forward_noalloc,

@@ -10,9 +10,23 @@
 
 #define MXATTN_API extern "C" __attribute__((visibility("default")))
 
+namespace mxattn {
+
+mxattn_status check_attention_shape(int B, int H, int N, int d, int kv_tile, int pnq, const float* O) {
+    if (B < 1 || H < 1 || N < 1 || O == nullptr) return MXATTN_ERR_INVALID;
+    if (pnq != 0 && pnq != 1) return MXATTN_ERR_INVALID;
+    if (d != 64 && d != 128) return MXATTN_ERR_UNSUPPORTED;
+    if (kv_tile != 64 && kv_tile != 128) return MXATTN_ERR_UNSUPPORTED;
+    if (N > kMaxAttentionN || static_cast<int64_t>(B) * H > (int64_t(1) << 31) / ((N + 127) / 128))
+        return MXATTN_ERR_UNSUPPORTED;
+    return MXATTN_OK;
+}
+
+}  // namespace mxattn
+
 namespace {
 
-constexpr int64_t kMaxN = int64_t(1) << 24;
+constexpr int64_t kMaxN = mxattn::kMaxAttentionN;
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -70,12 +84,9 @@ bool rule_qmax(mxattn_rule rule, float* qmax) {
 
 mxattn_status check_attention_args(int B, int H, int N, int d, int kv_tile, int pnq, const float* O, const void* ws,
                                    size_t ws_bytes, Layout* L) {
-    if (B < 1 || H < 1 || N < 1 || O == nullptr || ws == nullptr) return MXATTN_ERR_INVALID;
-    if (pnq != 0 && pnq != 1) return MXATTN_ERR_INVALID;
-    if (d != 64 && d != 128) return MXATTN_ERR_UNSUPPORTED;
-    if (kv_tile != 64 && kv_tile != 128) return MXATTN_ERR_UNSUPPORTED;
-    if (N > kMaxN || static_cast<int64_t>(B) * H > (int64_t(1) << 31) / ((N + 127) / 128))
-        return MXATTN_ERR_UNSUPPORTED;
+    if (ws == nullptr) return MXATTN_ERR_INVALID;
+    const mxattn_status st = mxattn::check_attention_shape(B, H, N, d, kv_tile, pnq, O);
+    if (st != MXATTN_OK) return st;
     if (!make_layout(B, H, N, d, L)) return MXATTN_ERR_INVALID;
     if (ws_bytes < L->total || !aligned(ws, 256) || !aligned(O, 16)) return MXATTN_ERR_INVALID;
     return MXATTN_OK;

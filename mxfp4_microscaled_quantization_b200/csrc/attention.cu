@@ -24,11 +24,17 @@
 //                      and the final O / l.
 //   warp 8 (one lane)  TMA producer: both Q tiles + scales once, then K and
 //                      V^T tiles (+ scales) into a kStages-deep ring.
-//   warp 9 (one lane)  MMA issuer: tcgen05.cp of E8M0 scales into TMEM and
-//                      tcgen05.mma kind::mxf4 block_scale, in the order
-//                      S_A(j), S_B(j), S_A(j+1) ... interleaved with
-//                      O_A += P_A V(j), O_B += P_B V(j).
-//   warps 10-11        idle (they complete the third warpgroup).
+//   warp 9 (one lane)  S issuer: tcgen05.cp of the Q and K scales into TMEM
+//                      and S_A(j) = Q_A K(j)^T, S_B(j) = Q_B K(j)^T
+//                      (tcgen05.mma kind::mxf4 block_scale) into the shared S
+//                      buffer, each as soon as the other tile has read the
+//                      buffer; it also allocates and frees TMEM.
+//   warp 10 (one lane) PV issuer: tcgen05.cp of the P and V^T scales and
+//                      O_A += P_A V(j), O_B += P_B V(j) as each P arrives.
+//                      With the S and PV products on two issuing threads, a
+//                      tile's next S never waits in program order behind the
+//                      other tile's P.
+//   warp 11            idle (it completes the third warpgroup).
 // The row sum under PNQ is produced by the tensor core itself: V^T gets one
 // extra row of ones (E2M1 1.0, scale 2^0) so O's column d accumulates
 // sum_j q_j -- exactly the quantized values that multiply V -- and is
@@ -72,9 +78,10 @@ struct Cfg {
     static constexpr int kRows = 128 * kTiles;        // query rows per CTA
     static constexpr int kSoftThreads = 128 * kTiles;
     static constexpr int kProducerWarp = 4 * kTiles;
-    static constexpr int kMmaWarp = 4 * kTiles + 1;
-    // A third, full warpgroup holds the producer and MMA warps (plus two idle
-    // warps) so registers can move between warpgroups with setmaxnreg.
+    static constexpr int kMmaWarp = 4 * kTiles + 1;  // S issuer (and TMEM allocator)
+    static constexpr int kPvWarp = 4 * kTiles + 2;   // PV issuer
+    // A third, full warpgroup holds the producer and the two MMA-issuing warps
+    // (plus one idle warp) so registers can move between warpgroups with setmaxnreg.
     static constexpr int kThreads = kSoftThreads + 128;
     // Launch: kThreads x kLaunchRegs registers (ptxas's cap for 12 warps, 3 per
     // sub-partition).  Split: softmax warpgroups kSoftRegs, the other kRoleRegs;
@@ -132,7 +139,8 @@ struct Cfg {
     //           s_full[kTiles], s_loaded[kTiles], p_full[kTiles], o_done[kTiles], drain
     static constexpr int kNumBars = 1 + 4 * kStages + 4 * kTiles + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kSmemUsed = kOffMisc + 16;
+    static constexpr int kOffNvTab = kOffMisc + 16;  // NVFP4: P's per-scale-code offsets, 2 x 128 fp32
+    static constexpr int kSmemUsed = kOffNvTab + (NV ? 1024 : 0);
     // >= 116 KB keeps one CTA per SM, so the 512-column TMEM allocation never waits
     static constexpr int kSmemBytes = (kSmemUsed + 1024 > 116 * 1024) ? kSmemUsed + 1024 : 116 * 1024;
 
@@ -160,17 +168,17 @@ struct KParams {
     int nkv;     // key tiles per head
     int groups;  // 128-row scale groups per head
     float kq;    // softmax_scale * log2(e)
-    // Block exponent of P in the log domain: e = sign * floor(sign * x + off) + add
-    // with x = log2 of the block's largest exponential.  Boundary Qmax < 8:
-    // sign = -1, off = log2(Qmax), add = 0, so e = ceil(x - log2 Qmax), the
-    // smallest e with 2^x <= Qmax * 2^e.  OCP (Qmax = 8): sign = +1, off = 0,
-    // add = -2, so e = floor(x) - 2 (floor of x itself, exact at integer x).
-    float e_sign;
-    float e_off;
-    int e_add;
+    // log2 Qmax of P's scale boundary when Qmax < 8 (the kernel's OCP form ignores it):
+    // block exponent e = ceil(x - log2 Qmax) with x the log2 of the block's largest exponential.
+    float log2q;
     // NVFP4: the second-level scales g of Q, K, V per (batch, head), [3][BH]
     const float* gs;
     int BH;
+    // NVFP4 P: per E4M3 scale code c (1..126), log2(2688 / value(c)) and
+    // (log2(2688 / value(c)) + 2) / 8, each computed in double and rounded once
+    // to fp32 (code 0, a block whose scale rounds to 0: 0 and 0.25).
+    float nv_off[128];
+    float nv_off8[128];
 };
 
 // Maximum of 32 values as a depth-4 tree of 3-input max instructions.
@@ -198,10 +206,10 @@ __device__ __forceinline__ uint64_t sf_desc(const void* p) {
     return smem_desc(smem_u32(p), 0, 128, kLayoutNone);
 }
 
-template <int D, int T, bool PNQ, bool NV>
+template <int D, int T, bool PNQ, bool NV, bool OCP>
 __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
     mxattn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, const KParams p) {
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ KParams p) {
     using C = Cfg<D, T, NV>;
     constexpr int S = C::kStages;
     constexpr int NT = C::kTiles;
@@ -230,6 +238,8 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
     uint64_t* bar_drain = bar_o_done + NT;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+    float* sNvOff = reinterpret_cast<float*>(smem + C::kOffNvTab);  // [128], NVFP4 only
+    float* sNvOff8 = sNvOff + 128;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -251,7 +261,7 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
             mbar_init(bar_p_full + t, 128);
             mbar_init(bar_o_done + t, 1);
         }
-        mbar_init(bar_drain, 1);
+        mbar_init(bar_drain, 2);  // one commit from each MMA-issuing thread
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -261,6 +271,12 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
         const int w = idx % (16 * (T / 2) / 4);
         const int row = D + w / (T / 8);
         reinterpret_cast<uint32_t*>(sV + s * C::kVStride + D * (T / 2))[w] = (row == D) ? 0x22222222u : 0u;
+    }
+    if constexpr (NV) {
+        for (int idx = tid; idx < 128; idx += C::kThreads) {
+            sNvOff[idx] = p.nv_off[idx];
+            sNvOff8[idx] = p.nv_off8[idx];
+        }
     }
     // Scale factors of V^T rows 128..255 (only used when D = 128): all 1 (E8M0 2^0, or E4M3 1.0).
     for (int idx = tid; idx < 128; idx += C::kThreads)
@@ -336,8 +352,8 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
             for (int j = v_issued - S < 0 ? 0 : v_issued - S; j < v_issued; ++j)
                 mbar_wait_bounded(bar_v_full + j % S, (j / S) & 1, no_abort, p.status, kTimeoutCode, kTimeoutNs);
             __syncwarp();
-    } else if (warp == C::kMmaWarp) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == C::kMmaWarp || warp == C::kPvWarp) {
+        // ------------------------------------------------------------ MMA issuers (S: warp 9, PV: warp 10)
             const uint32_t t_s = tbase + C::kColS;
             // Shared-memory descriptors of the first buffer of each operand; a buffer
             // b bytes further on is the descriptor plus b >> 4 (start-address field).
@@ -419,33 +435,43 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
                 __syncwarp();
                 return true;
             };
-            bool ok = wait(bar_q, 0);
-            if (ok) {
-                tc_fence_after_sync();
-                if (leader) {
-                    for (int t = 0; t < NT; ++t)
-                        for (int a = 0; a < C::kQAtoms; ++a)
-                            tc_cp_sf(tbase + C::kColQsf + 4 * C::kQAtoms * t + 4 * a,
-                                     sf_desc(sQsf + t * C::kQsfBytes + 512 * a));
-                    if (D == 128)
+            if (warp == C::kMmaWarp) {
+                // S issuer.  Order: S_A(0); S_B(0) once A has read the S buffer; then per
+                // key tile j: S_A(j) once B has read S_B(j-1), S_B(j) once A has read S_A(j).
+                bool ok = wait(bar_q, 0);
+                if (ok) {
+                    tc_fence_after_sync();
+                    if (leader) {
+                        for (int t = 0; t < NT; ++t)
+                            for (int a = 0; a < C::kQAtoms; ++a)
+                                tc_cp_sf(tbase + C::kColQsf + 4 * C::kQAtoms * t + 4 * a,
+                                         sf_desc(sQsf + t * C::kQsfBytes + 512 * a));
+                    }
+                    __syncwarp();
+                }
+                ok = ok && issue_s(0, 0);
+                ok = ok && wait(bar_s_loaded + 0, 0) && issue_s(1, 0);
+                for (int j = 1; ok && j < nkv; ++j) {
+                    ok = wait(bar_s_loaded + 1, (j - 1) & 1) && issue_s(0, j);
+                    ok = ok && wait(bar_s_loaded + 0, j & 1) && issue_s(1, j);
+                }
+            } else {
+                // PV issuer: the constant V^T scales of rows 128..255 once (d = 128), then
+                // O_A += P_A V(j) and O_B += P_B V(j) for every key tile, as each P arrives.
+                if (D == 128) {
+                    if (leader)
                         for (int slot = 0; slot < C::kSfSlots; ++slot)
                             for (int a = 0; a < C::kVAtoms; ++a)
                                 tc_cp_sf(tbase + C::kColVsf + 8 * C::kVAtoms * slot + 8 * a + 4, sf_desc(sVsfConst));
+                    __syncwarp();
                 }
-                __syncwarp();
+                for (int j = 0; j < nkv; ++j) {
+                    if (!issue_pv(0, j)) break;
+                    if (!issue_pv(1, j)) break;
+                }
             }
-            // Order: S_A(0); S_B(0) after A loaded; S_A(1) after B loaded; then per tile j:
-            // PV_A(j), S_B(j+1) (after A loaded S_A(j+1)), PV_B(j), S_A(j+2) (after B loaded S_B(j+1)).
-            ok = ok && issue_s(0, 0);
-            ok = ok && wait(bar_s_loaded + 0, 0) && issue_s(1, 0);
-            if (nkv > 1) ok = ok && wait(bar_s_loaded + 1, 0) && issue_s(0, 1);
-            for (int j = 0; ok && j < nkv; ++j) {
-                if (!issue_pv(0, j)) break;
-                if (j + 1 < nkv && !(wait(bar_s_loaded + 0, (j + 1) & 1) && issue_s(1, j + 1))) break;
-                if (!issue_pv(1, j)) break;
-                if (j + 2 < nkv && !(wait(bar_s_loaded + 1, (j + 1) & 1) && issue_s(0, j + 2))) break;
-            }
-            // Drain: wait for every MMA / copy the leader issued before TMEM is freed.
+            // Drain: wait for every MMA / copy both issuers made before TMEM is freed
+            // (bar_drain completes once each issuing thread's commit has arrived).
             if (leader) tc_commit(bar_drain);
             __syncwarp();
             int dummy = 0;
@@ -475,9 +501,7 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
             o_unit = __fmul_rn(6.f, p.gs[2 * p.BH + bh]);
         }
         const float kq8 = 0.125f * kq;  // exact: the stand-in's map of w onto [0, 1] scales by 1/8
-        const float e_sign = p.e_sign;
-        const float e_off = p.e_off;
-        const int e_add = p.e_add;
+        const float log2q = p.log2q;
         const int valid_last = p.N - (nkv - 1) * T;
         uint8_t* sPt = sP + t * C::kPBytes;
         uint8_t* sPsft = sPsf + t * C::kPsfBytes;
@@ -533,27 +557,29 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
                 // rounds to 0 holds values below 2.3e-6 and is left unscaled (all its codes are 0).
 #pragma unroll
                 for (int k = 0; k < NBM; ++k) {
-                    float sbv, l2;
-                    const uint32_t sb = nv_p_block_scale((bm[k] - m_new) * kq, sbv, l2);
-                    const bool scaled = sbv > 0.f;
-                    nbias[k] = fmaf(-m_new, kq, scaled ? 11.392317422778761f - l2 : 0.f);  // log2(2688 / sb)
-                    if constexpr (PNQ) nb8[k] = 0.125f * fmaf(-m_new, kq, scaled ? 13.392317422778761f - l2 : 2.f);
-                    back[k] = scaled ? sbv * (1.f / 2688.f) : 1.f;
+                    const uint32_t sb = nv_p_block_scale((bm[k] - m_new) * kq);
+                    nbias[k] = fmaf(-m_new, kq, sNvOff[sb]);                    // + log2(2688 / sb)
+                    if constexpr (PNQ) nb8[k] = fmaf(-m_new, kq8, sNvOff8[sb]);  // (nbias + 2) / 8
+                    if constexpr (!PNQ) {
+                        const float sbv = e4m3_decode(sb);
+                        back[k] = sbv > 0.f ? sbv * (1.f / 2688.f) : 1.f;
+                    }
                     sfw[k / 4] |= sb << (8 * (k % 4));
                 }
             } else {
                 // MXFP4 P: the block's largest exponential is 2^x with x = (bm - m_new) * kq; the
                 // scale rule is applied to it in the log domain (no exponential needed), and each
                 // element is then 2^(s*kq - (m*kq + e)), already divided by the block scale 2^e.
+                // bm - m_new is exactly 0 for the block holding the row max, so the OCP boundary
+                // at integer x is decided exactly there.
 #pragma unroll
                 for (int k = 0; k < NBM; ++k) {
-                    // x = (bm - m_new) * kq is exactly 0 for the block holding the row max, so
-                    // the OCP boundary at integer x is decided exactly there.
-                    const int e = p_block_exponent((bm[k] - m_new) * kq, e_sign, e_off, e_add);
-                    nbias[k] = -fmaf(m_new, kq, static_cast<float>(e));
-                    if constexpr (PNQ) nb8[k] = -0.125f * fmaf(m_new, kq, static_cast<float>(e - 2));
-                    back[k] = exp2_neg_int(-e);
-                    sfw[0] |= static_cast<uint32_t>(e + 127) << (8 * k);
+                    uint32_t byte;
+                    const float ef = p_block_exp<OCP>(bm[k] - m_new, kq, log2q, byte);
+                    nbias[k] = fmaf(-m_new, kq, -ef);                                      // -(m kq + e), one rounding
+                    if constexpr (PNQ) nb8[k] = fmaf(-m_new, kq8, fmaf(ef, -0.125f, 0.25f));  // (nbias + 2) / 8, one rounding
+                    if constexpr (!PNQ) back[k] = byte ? __uint_as_float(byte << 23) : __uint_as_float(0x00400000u);
+                    sfw[0] |= byte << (8 * k);
                 }
             }
             // Elements, 8 at a time (group gg: keys 8 gg .. 8 gg + 7, P block gg / (NV ? 2 : 4)).
@@ -679,7 +705,25 @@ bool encode_map(CUtensorMap* map, const void* base, uint64_t inner_bytes, uint64
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int T, bool PNQ, bool NV>
+// NVFP4 P: log2(2688 / value(c)) and (log2(2688 / value(c)) + 2) / 8 for every
+// E4M3 code c, computed in double and rounded once to fp32.  value(c): E4M3
+// (OCP FP8, bias 7) with exponent field c >> 3 and mantissa c & 7; code 0 (and
+// the unused NaN code 127) give 0 and 0.25, the offsets of an unscaled block.
+struct NvOffsets {
+    float off[128];
+    float off8[128];
+    NvOffsets() {
+        for (int c = 0; c < 128; ++c) {
+            const int E = c >> 3, M = c & 7;
+            const double v = (E == 0) ? std::ldexp(M / 8.0, -6) : std::ldexp(1.0 + M / 8.0, E - 7);
+            const double l = (c == 0 || c == 127) ? 0.0 : std::log2(2688.0 / v);
+            off[c] = static_cast<float>(l);
+            off8[c] = static_cast<float>((l + 2.0) / 8.0);
+        }
+    }
+};
+
+template <int D, int T, bool PNQ, bool NV, bool OCP>
 cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
     using C = Cfg<D, T, NV>;
     static bool attr_set = false;
@@ -687,10 +731,10 @@ cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
         // The setmaxnreg split assumes the launch allocates exactly kLaunchRegs per
         // thread; with fewer, the softmax warpgroups' increase could never be met.
         cudaFuncAttributes fa{};
-        cudaError_t e = cudaFuncGetAttributes(&fa, mxattn_fwd_kernel<D, T, PNQ, NV>);
+        cudaError_t e = cudaFuncGetAttributes(&fa, mxattn_fwd_kernel<D, T, PNQ, NV, OCP>);
         if (e != cudaSuccess) return e;
         if (fa.numRegs != static_cast<int>(C::kLaunchRegs)) return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, T, PNQ, NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(mxattn_fwd_kernel<D, T, PNQ, NV, OCP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
@@ -712,13 +756,18 @@ cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
     kp.nkv = (a.N + T - 1) / T;
     kp.groups = (a.N + 127) / 128;
     kp.kq = static_cast<float>(static_cast<double>(a.softmax_scale) * 1.4426950408889634);
-    kp.e_sign = a.qmax >= 8.f ? 1.f : -1.f;
-    kp.e_off = a.qmax >= 8.f ? 0.f : static_cast<float>(std::log2(static_cast<double>(a.qmax)));
-    kp.e_add = a.qmax >= 8.f ? -2 : 0;
+    kp.log2q = OCP ? 0.f : static_cast<float>(std::log2(static_cast<double>(a.qmax)));
     kp.gs = a.gs;
     kp.BH = static_cast<int>(a.BH);
+    if constexpr (NV) {
+        static const NvOffsets tab;
+        for (int c = 0; c < 128; ++c) {
+            kp.nv_off[c] = tab.off[c];
+            kp.nv_off8[c] = tab.off8[c];
+        }
+    }
     dim3 grid(static_cast<unsigned>(a.BH * kp.nq2));
-    mxattn_fwd_kernel<D, T, PNQ, NV><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, kp);
+    mxattn_fwd_kernel<D, T, PNQ, NV, OCP><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, kp);
     return cudaGetLastError();
 }
 
@@ -726,8 +775,11 @@ cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
 
 template <int D, int T>
 cudaError_t launch_pnq(const AttnArgs& a, cudaStream_t stream) {
-    if (a.nv) return a.pnq ? launch_impl<D, T, true, true>(a, stream) : launch_impl<D, T, false, true>(a, stream);
-    return a.pnq ? launch_impl<D, T, true, false>(a, stream) : launch_impl<D, T, false, false>(a, stream);
+    if (a.nv)
+        return a.pnq ? launch_impl<D, T, true, true, false>(a, stream) : launch_impl<D, T, false, true, false>(a, stream);
+    if (a.qmax >= 8.f)  // the OCP rule
+        return a.pnq ? launch_impl<D, T, true, false, true>(a, stream) : launch_impl<D, T, false, false, true>(a, stream);
+    return a.pnq ? launch_impl<D, T, true, false, false>(a, stream) : launch_impl<D, T, false, false, false>(a, stream);
 }
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t stream) {

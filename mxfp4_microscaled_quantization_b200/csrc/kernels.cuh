@@ -6,7 +6,18 @@
 
 #include <cstdint>
 
+#include "mxattn.h"
+
 namespace mxattn {
+
+// Largest sequence length the attention entry points accept.
+constexpr int64_t kMaxAttentionN = int64_t(1) << 24;
+
+// The argument checks every attention entry point runs first, in this order:
+// B, H, N >= 1 and O non-null (else MXATTN_ERR_INVALID), pnq in {0, 1}
+// (INVALID), d in {64, 128} and kv_tile in {64, 128} (MXATTN_ERR_UNSUPPORTED),
+// N <= kMaxAttentionN and the grid size (UNSUPPORTED).
+mxattn_status check_attention_shape(int B, int H, int N, int d, int kv_tile, int pnq, const float* O);
 
 // Row quantization of `ntensors` (1 or 2) bf16 tensors of shape [rows, cols].
 // regroup = 0: row-major scales; regroup = 1: rows are (bh, r < N), scales in

@@ -468,31 +468,35 @@ __device__ __forceinline__ float e4m3_decode(uint32_t b) {
     return f;
 }
 
-// Block exponent of an MXFP4 block of P from x = log2 of the block's largest
-// exponential (x <= 0; -inf for a block that is all masked), in the log
-// domain: e = sign * floor(sign * x + off) + add, with (sign, off, add) =
-// (-1, log2 Qmax, 0) for a boundary Qmax < 8, i.e. the smallest e with
-// 2^x <= Qmax * 2^e, and (+1, 0, -2) for OCP, i.e. floor(x) - 2.  Clamped to
-// [-127, ...]; |z| is clamped first so the round-down add stays exact.
-__device__ __forceinline__ int p_block_exponent(float x, float e_sign, float e_off, int e_add) {
-    float z = fmaf(e_sign, x, e_off);
-    z = fminf(fmaxf(z, -250.f), 250.f);
-    const int fl = static_cast<int>(__float_as_uint(__fadd_rd(z, 12582912.f)) - 0x4B400000u);
-    const int e = (e_sign > 0.f ? fl : -fl) + e_add;
-    return e < -127 ? -127 : e;
+// Block exponent e of an MXFP4 block of P, in the log domain, from d = bm - m
+// (the block's largest score minus the running maximum, <= 0; -inf for a
+// block that is all masked): x = d * kq is the log2 of the block's largest
+// exponential.  Scale boundary Qmax < 8 (UOS: 7.25): e = ceil(x - log2 Qmax),
+// the smallest e with 2^x <= Qmax * 2^e, formed as one rounding of
+// d * kq - log2 Qmax; OCP (Qmax = 8 with the OCP convention): e = floor(x) - 2,
+// with x rounded once, so x = 0 exactly for the block that holds the row
+// maximum.  The integer part comes from an add of 1.5 * 2^23 rounded up (ceil)
+// or down (floor), exact for |z| < 2^22; z is clamped first so e >= -127.
+// Returns e as an integer-valued float and sets `byte` to the E8M0 code e + 127.
+template <bool OCP>
+__device__ __forceinline__ float p_block_exp(float d, float kq, float log2q, uint32_t& byte) {
+    if constexpr (OCP) {
+        const float x = fmaxf(d * kq, -125.f);
+        const float t = __fadd_rd(x, 12582912.f);
+        byte = __float_as_uint(t) - 0x4B3FFF83u;  // floor(x) - 2 + 127
+        return t - 12582914.f;                    // floor(x) - 2
+    } else {
+        const float z = fmaxf(fmaf(d, kq, -log2q), -127.f);
+        const float t = __fadd_ru(z, 12582912.f);
+        byte = __float_as_uint(t) - 0x4B3FFF81u;  // ceil(z) + 127
+        return t - 12582912.f;                    // ceil(z)
+    }
 }
 
 // NVFP4 block of P from x = log2 of the block's largest exponential: the E4M3
-// scale sb = E4M3(2^x * 448), its value, and log2(sb) (meaningful only when
-// sb > 0).  log2(sb) is its fp32 exponent plus lg2.approx of its significand,
-// so lg2.approx only sees [1, 2), where its absolute error is smallest.
-__device__ __forceinline__ uint32_t nv_p_block_scale(float x, float& sbv, float& log2_sb) {
-    const uint32_t sb = e4m3_encode_sat(ex2_approx(x) * 448.f);
-    sbv = e4m3_decode(sb);
-    const uint32_t bits = __float_as_uint(sbv);
-    log2_sb = static_cast<float>(static_cast<int>(bits >> 23) - 127) +
-              lg2_approx(__uint_as_float((bits & 0x7FFFFFu) | 0x3F800000u));
-    return sb;
+// code of its scale, sb = E4M3(2^x * 448) (round to nearest even, saturating).
+__device__ __forceinline__ uint32_t nv_p_block_scale(float x) {
+    return e4m3_encode_sat(ex2_approx(x) * 448.f);
 }
 
 // Block exponent from the bfloat16 bit pattern of a block maximum (>= 0)

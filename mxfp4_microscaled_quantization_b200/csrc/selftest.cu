@@ -57,12 +57,11 @@ __global__ void __launch_bounds__(32) wait_selftest_kernel(int arrive, uint64_t 
 //               code-only stand-in / the FMA-pipe degree-5 exponential, each
 //               followed by cvt.rn.satfinite.e2m1x2;
 //   path 3:     in = x (log2 of a block's largest exponential), out = the
-//               MXFP4 block exponent for the scale boundary (e_sign, e_off, e_add);
+//               MXFP4 block exponent for the scale boundary (OCP, or log2 Qmax);
 //   path 4:     in = x, out = the NVFP4 block scale byte (E4M3 of 2^x * 448);
 //   path 5:     in = v, out = E2M1 code of v itself (the rounding step alone).
 __global__ void __launch_bounds__(256) p_selftest_kernel(int path, const float* __restrict__ in, int64_t n8,
-                                                         float e_sign, float e_off, int e_add,
-                                                         int32_t* __restrict__ out) {
+                                                         int ocp, float log2q, int32_t* __restrict__ out) {
     for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < n8;
          g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         float v[8];
@@ -89,13 +88,14 @@ __global__ void __launch_bounds__(256) p_selftest_kernel(int path, const float* 
             for (int i = 0; i < 8; ++i) out[8 * g + i] = static_cast<int32_t>((codes >> (4 * i)) & 0xFu);
         } else if (path == 3) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) out[8 * g + i] = p_block_exponent(v[i], e_sign, e_off, e_add);
+            for (int i = 0; i < 8; ++i) {
+                uint32_t byte;
+                const float e = ocp ? p_block_exp<true>(v[i], 1.f, 0.f, byte) : p_block_exp<false>(v[i], 1.f, log2q, byte);
+                out[8 * g + i] = static_cast<int32_t>(e);
+            }
         } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float sbv, l2;
-                out[8 * g + i] = static_cast<int32_t>(nv_p_block_scale(v[i], sbv, l2));
-            }
+            for (int i = 0; i < 8; ++i) out[8 * g + i] = static_cast<int32_t>(nv_p_block_scale(v[i]));
         }
     }
 }
@@ -111,12 +111,11 @@ MXATTN_API mxattn_status mxattn_p_selftest(int path, const float* in, int64_t n,
     if (in == nullptr || out == nullptr || (reinterpret_cast<uintptr_t>(in) & 3u) || (reinterpret_cast<uintptr_t>(out) & 3u))
         return MXATTN_ERR_INVALID;
     const bool ocp = qmax >= 8.f;
-    const float e_sign = ocp ? 1.f : -1.f;
-    const float e_off = ocp ? 0.f : static_cast<float>(std::log2(static_cast<double>(qmax)));
+    const float log2q = ocp ? 0.f : static_cast<float>(std::log2(static_cast<double>(qmax)));
     const int64_t n8 = n / 8;
     const int grid = static_cast<int>(n8 / 256 + 1 < 4096 ? n8 / 256 + 1 : 4096);
-    mxattn::p_selftest_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(path, in, n8, e_sign, e_off,
-                                                                                         ocp ? -2 : 0, out);
+    mxattn::p_selftest_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(path, in, n8, ocp ? 1 : 0,
+                                                                                         log2q, out);
     return cudaGetLastError() == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
 }
 

@@ -58,6 +58,11 @@ def lib() -> ctypes.CDLL:
         L.mxattn_forward_quantized.restype = i32
         L.mxattn_forward_noalloc.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, ctypes.c_float, P, P]
         L.mxattn_forward_noalloc.restype = i32
+        L.mxattn_forward_host_workspace_size.argtypes = [i32, i32, i32, i32, P, i32]
+        L.mxattn_forward_host_workspace_size.restype = u64
+        L.mxattn_forward_host.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, ctypes.c_float, P, P, P, P, P, P,
+                                          u64, P, i32, P]
+        L.mxattn_forward_host.restype = i32
         f32 = ctypes.c_float
         L.mxattn_quantize_qmax.argtypes = [P, i64, i64, f32, P, P, P]
         L.mxattn_quantize_qmax.restype = i32
@@ -271,10 +276,16 @@ def mxattn_forward_noalloc(q, k, v, kv_tile=128, pnq=True, rule="uos", softmax_s
         raise ValueError("q, k, v must have the same shape [B, H, N, d]")
     if out is None:
         out = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
-    _check(lib().mxattn_forward_noalloc(_cuda(q, "q", torch.bfloat16), _cuda(k, "k", torch.bfloat16),
-                                        _cuda(v, "v", torch.bfloat16), B, H, N, d, kv_tile, 1 if pnq else 0,
-                                        _rule(rule), float(softmax_scale), _cuda(out, "out", torch.float32),
-                                        _stream(stream)), "mxattn_forward_noalloc")
+    for name, t in (("k", k), ("v", v), ("out", out)):
+        if t.device != q.device:
+            raise ValueError(f"{name} is on {t.device}, q on {q.device}: all tensors must be on one device")
+    # The library's scratch is the one on the current device: make q's device current for the call.
+    with torch.cuda.device(q.device):
+        s = _stream(torch.cuda.current_stream(q.device) if stream is None else stream)
+        _check(lib().mxattn_forward_noalloc(_cuda(q, "q", torch.bfloat16), _cuda(k, "k", torch.bfloat16),
+                                            _cuda(v, "v", torch.bfloat16), B, H, N, d, kv_tile, 1 if pnq else 0,
+                                            _rule(rule), float(softmax_scale), _cuda(out, "out", torch.float32),
+                                            s), "mxattn_forward_noalloc")
     return out
 
 
@@ -329,22 +340,10 @@ def mxattn_status_string(status: int) -> str:
     return status_string(status)
 
 
-_side_streams = {}
-
-
-def _copy_streams(device):
-    """Two side streams per device for the host<->device copies of attention_from_host."""
-    key = torch.device(device).index
-    if key not in _side_streams:
-        _side_streams[key] = (torch.cuda.Stream(device), torch.cuda.Stream(device))
-    return _side_streams[key]
-
-
 def host_groups(BH: int, chunks: int = 16):
-    """Sizes of the (batch, head) groups attention_from_host pipelines by
-    default: `chunks` groups, the first and the last of one slice each (the
-    copy to the device of the first group and the copy back of the last are
-    the only transfers nothing else overlaps), the rest as equal as possible."""
+    """Sizes of the (batch, head) groups mxattn_forward_host pipelines by default
+    (the library's schedule, restated): `chunks` groups, the first and the last
+    of one slice each, the rest as equal as possible."""
     if BH <= 0:
         return []
     n = max(1, min(int(chunks), BH))
@@ -355,20 +354,27 @@ def host_groups(BH: int, chunks: int = 16):
     return [1] + [mid // k + (1 if i < mid % k else 0) for i in range(k)] + [1]
 
 
+def _group_args(groups, chunks):
+    if groups is None:
+        return None, int(chunks)
+    arr = (ctypes.c_int * len(groups))(*[int(g) for g in groups])
+    return arr, len(groups)
+
+
+def forward_host_workspace_size(B, H, N, d, chunks=16, groups=None) -> int:
+    arr, n = _group_args(groups, chunks)
+    return int(lib().mxattn_forward_host_workspace_size(B, H, N, d, arr, n))
+
+
 def attention_from_host(q_host, k_host, v_host, kv_tile=128, pnq=True, rule="uos", softmax_scale=0.0,
                         device_buffers=None, out_host=None, stream=None, chunks=16, groups=None):
-    """End-to-end call with host tensors: q, k, v (pinned host bf16 [B, H, N, d])
-    to the device, mxattn_forward, O back into `out_host` (pinned fp32).
-
-    The (batch, head) slices are processed in groups (`groups`: their sizes,
-    summing to B*H; default host_groups(B*H, chunks)), pipelined over three
-    streams: the copy of group i+1 to the device and of group i-1 back to the
-    host overlap the attention of group i (heads are independent, so each
-    group is one mxattn_forward call on a contiguous slice).  The work is
-    ordered on `stream` (default: the current stream): everything, including
-    the last copy back, is done when `stream` reaches the point after this call.
+    """End-to-end call with host tensors through mxattn_forward_host: q, k, v
+    (pinned host bf16 [B, H, N, d]) to the device, the attention, O back into
+    `out_host` (pinned fp32), pipelined over (batch, head) groups inside the
+    library (`groups`: their sizes, summing to B*H; default: `chunks` groups).
+    The work is ordered on `stream` (default: the current stream).
     `device_buffers` = (q, k, v, out, workspace) device tensors to reuse; the
-    workspace needs only the size of the largest group."""
+    workspace needs forward_host_workspace_size(...) bytes."""
     B, H, N, d = q_host.shape
     BH = B * H
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -380,42 +386,27 @@ def attention_from_host(q_host, k_host, v_host, kv_tile=128, pnq=True, rule="uos
     qd, kd, vd, od, ws = device_buffers
     if out_host is None:
         out_host = torch.empty((B, H, N, d), dtype=torch.float32, pin_memory=True)
-    sizes = host_groups(BH, chunks) if groups is None else [int(g) for g in groups]
-    if BH and (sum(sizes) != BH or min(sizes) < 1):
-        raise ValueError(f"groups {sizes} must be positive and sum to B*H = {BH}")
+    if groups is not None:
+        sizes = [int(g) for g in groups]
+        if BH and (sum(sizes) != BH or min(sizes) < 1):
+            raise ValueError(f"groups {sizes} must be positive and sum to B*H = {BH}")
+    arr, n = _group_args(groups, chunks)
     if ws is None:
-        ws = new_workspace(1, max(sizes, default=1), N, d, dev)
-    compute = torch.cuda.current_stream(dev) if stream is None else stream
-    h2d, d2h = _copy_streams(dev)
-    h2d.wait_stream(compute)  # the device buffers may still be in use by earlier work on `stream`
-    d2h.wait_stream(compute)
-    flat = lambda t: t.view(BH, N, d)  # noqa: E731
-    qh, kh, vh, oh = flat(q_host), flat(k_host), flat(v_host), flat(out_host)
-    qf, kf, vf, of = flat(qd), flat(kd), flat(vd), flat(od)
-    last = None
-    c0 = 0
-    for size in sizes:
-        sl = slice(c0, c0 + size)
-        c0 += size
-        with torch.cuda.stream(h2d):
-            qf[sl].copy_(qh[sl], non_blocking=True)
-            kf[sl].copy_(kh[sl], non_blocking=True)
-            vf[sl].copy_(vh[sl], non_blocking=True)
-            loaded = torch.cuda.Event()
-            loaded.record(h2d)
-        compute.wait_event(loaded)
-        nh = sl.stop - sl.start
-        mxattn_forward(qf[sl].view(1, nh, N, d), kf[sl].view(1, nh, N, d), vf[sl].view(1, nh, N, d), kv_tile, pnq,
-                       rule, softmax_scale, of[sl].view(1, nh, N, d), ws, compute)
-        done = torch.cuda.Event()
-        done.record(compute)
-        d2h.wait_event(done)
-        with torch.cuda.stream(d2h):
-            oh[sl].copy_(of[sl], non_blocking=True)
-            last = torch.cuda.Event()
-            last.record(d2h)
-    if last is not None:
-        compute.wait_event(last)
+        need = int(lib().mxattn_forward_host_workspace_size(B, H, N, d, arr, n))
+        if need == 0:
+            raise MxattnError(1, "mxattn_forward_host_workspace_size")
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    for name, t in (("q", q_host), ("k", k_host), ("v", v_host), ("out", out_host)):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host tensor")
+    if q_host.dtype != torch.bfloat16 or out_host.dtype != torch.float32:
+        raise ValueError("q, k, v must be bfloat16 and out float32")
+    hp = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    _check(lib().mxattn_forward_host(hp(q_host), hp(k_host), hp(v_host), B, H, N, d, kv_tile, 1 if pnq else 0,
+                                     _rule(rule), float(softmax_scale), hp(out_host), _cuda(qd, "q_dev"),
+                                     _cuda(kd, "k_dev"), _cuda(vd, "v_dev"), _cuda(od, "o_dev", torch.float32),
+                                     _cuda(ws, "workspace"), ws.numel(), arr, n, _stream(stream)),
+           "mxattn_forward_host")
     return out_host
 
 

@@ -81,6 +81,34 @@ def test_forward_rejects_bad_arguments_before_launching(L):
     assert L.mxattn_forward_quantized(*q, 1, 1, 256, 64, 96, 1, 1, ctypes.c_float(0), fake, fake, ws_ok, None) == 2
 
 
+def test_forward_host_rejects_bad_arguments_before_launching(L):
+    """mxattn_forward_host checks everything before it creates a stream or copies a byte."""
+    fake = _p(1 << 20)
+    ws = mx.forward_host_workspace_size(1, 4, 256, 64)
+    ok = dict(d=64, t=64, pnq=1, rule=1, N=256, H=4, o=fake, dev=fake, ws=fake, wsb=ws, groups=None, ng=0)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return L.mxattn_forward_host(fake, fake, fake, 1, a["H"], a["N"], a["d"], a["t"], a["pnq"], a["rule"],
+                                     ctypes.c_float(0.0), a["o"], a["dev"], fake, fake, fake, a["ws"], a["wsb"],
+                                     a["groups"], a["ng"], None)
+    assert call(d=96) == 2
+    assert call(t=32) == 2
+    assert call(N=(1 << 24) + 1, wsb=1 << 40) == 2
+    assert call(pnq=2) == 1
+    assert call(rule=5) == 1
+    assert call(o=None) == 1
+    assert call(dev=None) == 1
+    assert call(dev=_p((1 << 20) + 4)) == 1          # misaligned staging buffer
+    assert call(ws=_p((1 << 20) + 16)) == 1          # misaligned workspace
+    assert call(wsb=ws - 1) == 1                      # workspace too small for the largest group
+    bad = (ctypes.c_int * 2)(3, 2)                     # sums to 5, B*H = 4
+    assert call(groups=bad, ng=2) == 1
+    zero = (ctypes.c_int * 2)(4, 0)
+    assert call(groups=zero, ng=2) == 1
+    assert call(ng=-1) == 1
+
+
 def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(mx, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(mx, "_lib", None)
@@ -168,8 +196,9 @@ def test_header_compiles_as_c_and_links(L, tmp_path):
         "int main(void) {\n"
         "  size_t ws = mxattn_workspace_size(1, 40, 32760, 128);\n"
         "  size_t nv = mxattn_nvfp4_workspace_size(1, 40, 32760, 128);\n"
+        "  size_t hw = mxattn_forward_host_workspace_size(1, 40, 32760, 128, 0, 0);\n"
         "  mxattn_status st = mxattn_quantize(0, 4, 48, MXATTN_RULE_UOS, 0, 0, 0);\n"
-        "  printf(\"%zu %zu %d %s\\n\", ws, nv, (int)st, mxattn_status_string(st));\n"
+        "  printf(\"%zu %zu %d %s %zu\\n\", ws, nv, (int)st, mxattn_status_string(st), hw);\n"
         "  return 0;\n}\n")
     exe = tmp_path / "abi"
     libdir = os.path.dirname(mx.LIB_PATH)
@@ -179,4 +208,5 @@ def test_header_compiles_as_c_and_links(L, tmp_path):
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     assert int(out[0]) == mx.mxattn_workspace_size(1, 40, 32760, 128)
     assert int(out[1]) == mx.nvfp4_workspace_size(1, 40, 32760, 128)
-    assert out[2] == "1" and " ".join(out[3:]) == mx.status_string(1)
+    assert out[2] == "1" and " ".join(out[3:-1]) == mx.status_string(1)
+    assert int(out[-1]) == mx.forward_host_workspace_size(1, 40, 32760, 128)

@@ -7,18 +7,17 @@ Criteria (MXAttention abstract, "MXAttention: Data-Free Optimal Scaling and
 Pre-Normalization Quantization for MXFP4 Attention"; the target's tolerance
 for O is rel-Frobenius <= 1e-3 and max-abs <= 2e-2):
   - Q, K, V^T codes and scales: bit for bit;
-  - O: max-abs <= 2e-2 everywhere, and rel-Frobenius <= 1e-3 over the rows
-    that no P decision flip touched.  The kernel decides P's codes in fp32
-    and the oracle in fp64, so an exponential within fp32 rounding of a
-    rounding point may round the other way.  That moves one weight of one
-    row by one E2M1 step: that row's error jumps from about 1e-7 to up to a
-    few percent while every other row stays near 1e-7.  Rows above 1e-5
-    relative error count as touched; at most 1 % of the rows may be (measured
-    rate: well under 0.1 %).  Without PNQ the row sum adds unquantized fp32
-    exponentials whose exponents carry the fp32 rounding of m * kq, so rows with
-    large scores (|m kq| in the hundreds) differ from the fp64 oracle by a common
-    factor up to ln 2 * ulp(|m kq|); that bound is added to the row threshold
-    there.
+  - O: max-abs <= 2e-2 and rel-Frobenius <= 1e-3 over every checked row of
+    every case, no row excluded.
+As a printed diagnostic only, each case reports how many rows a P decision
+flip touched.  The kernel decides P's codes in fp32 and the oracle in fp64,
+so an exponential within fp32 rounding of a rounding point may round the
+other way; that moves one weight of one row by one E2M1 step, so that row's
+error jumps from about 1e-7 to as much as a few percent.  A row counts as
+touched above 1e-5 relative error; without PNQ the row sum adds unquantized
+fp32 exponentials whose exponents carry the fp32 rounding of m * kq, so rows
+with large scores (|m kq| in the hundreds) differ from the fp64 oracle by a
+common factor up to ln 2 * ulp(|m kq|), which is added to that threshold.
 """
 import numpy as np
 import pytest
@@ -84,18 +83,16 @@ def _exponent_bias_bound(Q, K, rows, scale, rule=None):
 
 
 def _check_o(O, R, what, row_bound=None):
-    """max-abs <= 2e-2; rows above 1e-5 relative error (plus row_bound, the fp32
-    exponent-bias bound of PNQ-off rows) count as touched by a P decision flip:
-    at most 1 %; rel-Frobenius <= 1e-3 over the others."""
+    """max-abs <= 2e-2 and rel-Frobenius <= 1e-3 over all rows; returns the number of
+    rows a P decision flip touched (relative error above 1e-5, plus row_bound, the fp32
+    exponent-bias bound of PNQ-off rows) as a diagnostic."""
     assert np.all(np.isfinite(O)), what
     mabs = float(np.max(np.abs(O - R)))
-    assert mabs <= 2e-2, f"{what}: max-abs {mabs:.3e}"
+    rel = float(np.linalg.norm(O - R) / np.linalg.norm(R))
     rows = np.linalg.norm(O - R, axis=-1) / np.maximum(np.linalg.norm(R, axis=-1), 1e-30)
     touched = rows > 1e-5 + (0.0 if row_bound is None else row_bound)
-    assert touched.mean() <= 0.01, f"{what}: {touched.sum()} of {touched.size} rows above 1e-5"
-    keep = ~touched
-    rel = np.linalg.norm((O - R)[keep]) / np.linalg.norm(R[keep])
-    assert rel <= 1e-3, f"{what}: rel-Frobenius {rel:.3e} over untouched rows"
+    assert mabs <= 2e-2, f"{what}: max-abs {mabs:.3e} ({touched.sum()} rows touched by P flips)"
+    assert rel <= 1e-3, f"{what}: rel-Frobenius {rel:.3e} over all rows ({touched.sum()} rows touched by P flips)"
     return int(touched.sum()), rel, mabs
 
 

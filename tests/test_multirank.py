@@ -129,3 +129,25 @@ def test_sequence_layout_transforms_are_identity_on_one_rank():
 
     x = torch.arange(2 * 4 * 6 * 8, dtype=torch.float32).reshape(2, 4, 6, 8)
     assert ulysses.seq_to_head(x) is x and ulysses.head_to_seq(x) is x
+
+
+def test_bench_gpus_flag_starts_its_own_ranks():
+    """`bench.py --gpus 2` outside torchrun starts two ranks on this node itself
+    (here the reference arm, which runs on the host: rank 0 times the oracle and
+    prints the one JSON line, rank 1 exits without work)."""
+    import json
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR",
+                                                            "MASTER_PORT")}
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--impl", "reference",
+                          "--steps", "1", "--warmup", "3", "--ref-step-budget", "0.2"], capture_output=True,
+                         text=True, env=env, cwd=root, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["steps"] == 1
+    assert line["config"] == bench.config_dict(bench.WORKLOAD, 2, "replicas")
