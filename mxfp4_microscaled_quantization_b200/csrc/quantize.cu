@@ -15,8 +15,9 @@
 //    order the tensor core reads scale factors).
 //  * quantize_vt_kernel: V blocks of 32 consecutive tokens per channel,
 //    written transposed (V^T, tokens contiguous): a CTA stages 128 tokens x d
-//    channels in shared memory and each thread quantizes (channel, block)
-//    columns from there.
+//    channels in shared memory and each thread quantizes the blocks of a pair
+//    of channels over a run of tokens from there (one 32-bit shared-memory
+//    read per token for both channels).
 //  * regroup_sf_kernel: row-major scales -> the 128-row regrouped order.
 #include <cuda_runtime.h>
 
@@ -145,67 +146,96 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_grouped_kernel(Ro
             reinterpret_cast<const uint4*>(sf)[threadIdx.x];
 }
 
-// V^T quantization: grid (G token groups of 128, BH), D threads.  The CTA stages
-// 128 tokens x D channels (bf16) in shared memory; thread `ch` then quantizes
-// the four 32-token blocks of its channel and writes 64 contiguous code bytes.
+// V^T quantization: grid (G token groups of 128, BH), 128 threads.  The CTA
+// stages 128 tokens x D channels (bf16) in shared memory.  Each thread then
+// owns a pair of adjacent channels over a run of 256 / D * 16 tokens (64 for
+// D = 128, 32 for D = 64): it reads its two channels of a token as one 32-bit
+// word (a warp reads 128 contiguous bytes of a token row), quantizes the 32-
+// token blocks of both channels, and writes each channel's codes for its run
+// as contiguous 16-byte stores.
 template <int D>
-__global__ void __launch_bounds__(D) quantize_vt_kernel(const uint16_t* __restrict__ v, int N, int npad, uint32_t sf_thresh,
-                                                        int regroup, int groups, uint8_t* __restrict__ codes_t,
-                                                        uint8_t* __restrict__ scales_t) {
+__global__ void __launch_bounds__(128) quantize_vt_kernel(const uint16_t* __restrict__ v, int N, int npad, uint32_t sf_thresh,
+                                                          int regroup, int groups, uint8_t* __restrict__ codes_t,
+                                                          uint8_t* __restrict__ scales_t) {
+    constexpr int kPairs = D / 2;             // channel pairs
+    constexpr int kRuns = 128 / kPairs;       // token runs per 128-token group (2 or 4)
+    constexpr int kRun = 128 / kRuns;         // tokens per run (64 or 32)
+    constexpr int kBlocks = kRun / 32;        // 32-token blocks per run (2 or 1)
     __shared__ __align__(16) uint16_t tile[128 * D];
     const int g = blockIdx.x;
     const int64_t bh = blockIdx.y;
     const int t0 = g * 128;
-    const int ch = threadIdx.x;
+    const int tid = threadIdx.x;
     constexpr int kChunksPerRow = D / 8;
-    constexpr int kPerThread = 128 * kChunksPerRow / D;  // 16 loads of 16 bytes in flight
+    constexpr int kPerThread = 128 * kChunksPerRow / 128;  // 16-byte loads in flight per thread
     uint4 val[kPerThread];
 #pragma unroll
     for (int u = 0; u < kPerThread; ++u) {
-        const int c = ch + u * D;
+        const int c = tid + u * 128;
         const int t = c / kChunksPerRow;
         val[u] = (t0 + t < N) ? __ldcs(reinterpret_cast<const uint4*>(v + (bh * N + t0 + t) * D) + (c % kChunksPerRow))
                               : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int u = 0; u < kPerThread; ++u) reinterpret_cast<uint4*>(tile)[ch + u * D] = val[u];
+    for (int u = 0; u < kPerThread; ++u) reinterpret_cast<uint4*>(tile)[tid + u * 128] = val[u];
     __syncthreads();
-    uint32_t sfword = 0;
-    uint8_t* rowp = codes_t + (bh * D + ch) * static_cast<int64_t>(npad / 2);
+    const int cp = tid % kPairs;   // channels 2 cp, 2 cp + 1
+    const int run = tid / kPairs;  // tokens [run * kRun, run * kRun + kRun) of the group
+    const uint32_t* tile32 = reinterpret_cast<const uint32_t*>(tile);
+    uint32_t sfbytes[2] = {0u, 0u};  // per channel: the scale bytes of this run's blocks
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        uint32_t amax = 0;
-        uint32_t raw[32];
+    for (int b = 0; b < kBlocks; ++b) {
+        uint32_t raw[32];  // token i of the block: channel 2 cp in the low half, 2 cp + 1 in the high half
+        uint32_t amax0 = 0, amax1 = 0;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            raw[i] = tile[(32 * k + i) * D + ch];
-            amax = max(amax, raw[i] & 0x7FFFu);
+            raw[i] = tile32[(run * kRun + 32 * b + i) * kPairs + cp];
+            amax0 = max(amax0, raw[i] & 0x7FFFu);
+            amax1 = max(amax1, (raw[i] >> 16) & 0x7FFFu);
         }
-        const int e = block_exponent_bf16(amax, sf_thresh);
-        const float sc = exp2_neg_int(e);
-        uint32_t words[4];
+        const int tb = t0 + run * kRun + 32 * b;  // first token of the block
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            float f[8];
+        for (int h = 0; h < 2; ++h) {
+            const int e = block_exponent_bf16(h ? amax1 : amax0, sf_thresh);
+            const float sc = exp2_neg_int(e);
+            uint32_t words[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(raw[8 * w + i] << 16) * sc;
-            words[w] = pack_e2m1x8(f);
+            for (int w = 0; w < 4; ++w) {
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    f[i] = __uint_as_float(h ? (raw[8 * w + i] & 0xFFFF0000u) : (raw[8 * w + i] << 16)) * sc;
+                words[w] = pack_e2m1x8(f);
+            }
+            const int ch = 2 * cp + h;
+            uint8_t* rowp = codes_t + (bh * D + ch) * static_cast<int64_t>(npad / 2);
+            if (tb < npad) *reinterpret_cast<uint4*>(rowp + tb / 2) = make_uint4(words[0], words[1], words[2], words[3]);
+            const uint32_t sbyte = static_cast<uint32_t>(e + 127);
+            sfbytes[h] |= sbyte << (8 * b);
+            if (!regroup && tb < npad) scales_t[(bh * D + ch) * static_cast<int64_t>(npad / 32) + tb / 32] = sbyte;
         }
-        const int tb = t0 + 32 * k;  // first token of the block
-        if (tb < npad) *reinterpret_cast<uint4*>(rowp + tb / 2) = make_uint4(words[0], words[1], words[2], words[3]);
-        const uint32_t sbyte = static_cast<uint32_t>(e + 127);
-        sfword |= sbyte << (8 * k);
-        if (!regroup && tb < npad) scales_t[(bh * D + ch) * static_cast<int64_t>(npad / 32) + tb / 32] = sbyte;
     }
     if (regroup) {
-        // group g of 128 tokens; channel ch plays the role of the row
+        // group g of 128 tokens; channel ch plays the role of the row, block k of the
+        // group its byte k: this run's blocks are bytes run * kBlocks ...
         uint8_t* grp = scales_t + (bh * groups + g) * 512;
-        *reinterpret_cast<uint32_t*>(grp + (ch & 31) * 16 + (ch >> 5) * 4) = sfword;
-        if (D < 128) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int ch = 2 * cp + h;
+            uint8_t* word = grp + (ch & 31) * 16 + (ch >> 5) * 4 + run * kBlocks;
+            if constexpr (kBlocks == 2)
+                *reinterpret_cast<uint16_t*>(word) = static_cast<uint16_t>(sfbytes[h]);
+            else
+                *word = static_cast<uint8_t>(sfbytes[h]);
+        }
+        if (D < 128 && run == 0) {
             // channel rows D..127 of the group: scale 2^0, so the extra ones-row the
             // attention kernel appends to V^T (row D) is read with unit scale
-            const int c2 = ch + D;
-            *reinterpret_cast<uint32_t*>(grp + (c2 & 31) * 16 + (c2 >> 5) * 4) = 0x7F7F7F7Fu;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int c2 = 2 * cp + h + D;
+                *reinterpret_cast<uint32_t*>(grp + (c2 & 31) * 16 + (c2 >> 5) * 4) = 0x7F7F7F7Fu;
+            }
         }
     }
 }
@@ -289,8 +319,8 @@ cudaError_t launch_quantize_vt(const void* v, int64_t BH, int N, int d, uint32_t
         quantize_vt_kernel<128><<<grid, 128, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, sf_thresh, regroup,
                                                            groups, codes_t, scales_t);
     else
-        quantize_vt_kernel<64><<<grid, 64, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, sf_thresh, regroup, groups,
-                                                         codes_t, scales_t);
+        quantize_vt_kernel<64><<<grid, 128, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, sf_thresh, regroup,
+                                                          groups, codes_t, scales_t);
     return cudaGetLastError();
 }
 
