@@ -139,8 +139,7 @@ struct Cfg {
     //           s_full[kTiles], s_loaded[kTiles], p_full[kTiles], o_done[kTiles], drain
     static constexpr int kNumBars = 1 + 4 * kStages + 4 * kTiles + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kOffNvTab = kOffMisc + 16;  // NVFP4: P's per-scale-code offsets, 2 x 128 fp32
-    static constexpr int kSmemUsed = kOffNvTab + (NV ? 1024 : 0);
+    static constexpr int kSmemUsed = kOffMisc + 16;
     // >= 116 KB keeps one CTA per SM, so the 512-column TMEM allocation never waits
     static constexpr int kSmemBytes = (kSmemUsed + 1024 > 116 * 1024) ? kSmemUsed + 1024 : 116 * 1024;
 
@@ -174,11 +173,6 @@ struct KParams {
     // NVFP4: the second-level scales g of Q, K, V per (batch, head), [3][BH]
     const float* gs;
     int BH;
-    // NVFP4 P: per E4M3 scale code c (1..126), log2(2688 / value(c)) and
-    // (log2(2688 / value(c)) + 2) / 8, each computed in double and rounded once
-    // to fp32 (code 0, a block whose scale rounds to 0: 0 and 0.25).
-    float nv_off[128];
-    float nv_off8[128];
 };
 
 // Maximum of 32 values as a depth-4 tree of 3-input max instructions.
@@ -238,8 +232,6 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
     uint64_t* bar_drain = bar_o_done + NT;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
-    float* sNvOff = reinterpret_cast<float*>(smem + C::kOffNvTab);  // [128], NVFP4 only
-    float* sNvOff8 = sNvOff + 128;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -271,12 +263,6 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
         const int w = idx % (16 * (T / 2) / 4);
         const int row = D + w / (T / 8);
         reinterpret_cast<uint32_t*>(sV + s * C::kVStride + D * (T / 2))[w] = (row == D) ? 0x22222222u : 0u;
-    }
-    if constexpr (NV) {
-        for (int idx = tid; idx < 128; idx += C::kThreads) {
-            sNvOff[idx] = p.nv_off[idx];
-            sNvOff8[idx] = p.nv_off8[idx];
-        }
     }
     // Scale factors of V^T rows 128..255 (only used when D = 128): all 1 (E8M0 2^0, or E4M3 1.0).
     for (int idx = tid; idx < 128; idx += C::kThreads)
@@ -558,12 +544,14 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < NBM; ++k) {
                     const uint32_t sb = nv_p_block_scale((bm[k] - m_new) * kq);
-                    nbias[k] = fmaf(-m_new, kq, sNvOff[sb]);                    // + log2(2688 / sb)
-                    if constexpr (PNQ) nb8[k] = fmaf(-m_new, kq8, sNvOff8[sb]);  // (nbias + 2) / 8
-                    if constexpr (!PNQ) {
-                        const float sbv = e4m3_decode(sb);
-                        back[k] = sbv > 0.f ? sbv * (1.f / 2688.f) : 1.f;
-                    }
+                    const float sbv = e4m3_decode(sb);
+                    // log2(2688 / sbv) split as an exact integer plus a fraction rounded once:
+                    // ei = 138 - (biased fp32 exponent of sbv), fr = log2(1.3125) - log2(significand).
+                    float ei, fr;
+                    nv_p_scale_log2_parts(sbv, ei, fr);
+                    nbias[k] = fmaf(-m_new, kq, sb ? fr + ei : 0.f);
+                    if constexpr (PNQ) nb8[k] = fmaf(-m_new, kq8, sb ? fmaf(fr, 0.125f, fmaf(ei, 0.125f, 0.25f)) : 0.25f);
+                    if constexpr (!PNQ) back[k] = sb ? sbv * (1.f / 2688.f) : 1.f;
                     sfw[k / 4] |= sb << (8 * (k % 4));
                 }
             } else {
@@ -705,24 +693,6 @@ bool encode_map(CUtensorMap* map, const void* base, uint64_t inner_bytes, uint64
     return r == CUDA_SUCCESS;
 }
 
-// NVFP4 P: log2(2688 / value(c)) and (log2(2688 / value(c)) + 2) / 8 for every
-// E4M3 code c, computed in double and rounded once to fp32.  value(c): E4M3
-// (OCP FP8, bias 7) with exponent field c >> 3 and mantissa c & 7; code 0 (and
-// the unused NaN code 127) give 0 and 0.25, the offsets of an unscaled block.
-struct NvOffsets {
-    float off[128];
-    float off8[128];
-    NvOffsets() {
-        for (int c = 0; c < 128; ++c) {
-            const int E = c >> 3, M = c & 7;
-            const double v = (E == 0) ? std::ldexp(M / 8.0, -6) : std::ldexp(1.0 + M / 8.0, E - 7);
-            const double l = (c == 0 || c == 127) ? 0.0 : std::log2(2688.0 / v);
-            off[c] = static_cast<float>(l);
-            off8[c] = static_cast<float>((l + 2.0) / 8.0);
-        }
-    }
-};
-
 template <int D, int T, bool PNQ, bool NV, bool OCP>
 cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
     using C = Cfg<D, T, NV>;
@@ -759,13 +729,6 @@ cudaError_t launch_impl(const AttnArgs& a, cudaStream_t stream) {
     kp.log2q = OCP ? 0.f : static_cast<float>(std::log2(static_cast<double>(a.qmax)));
     kp.gs = a.gs;
     kp.BH = static_cast<int>(a.BH);
-    if constexpr (NV) {
-        static const NvOffsets tab;
-        for (int c = 0; c < 128; ++c) {
-            kp.nv_off[c] = tab.off[c];
-            kp.nv_off8[c] = tab.off8[c];
-        }
-    }
     dim3 grid(static_cast<unsigned>(a.BH * kp.nq2));
     mxattn_fwd_kernel<D, T, PNQ, NV, OCP><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, kp);
     return cudaGetLastError();

@@ -499,6 +499,19 @@ __device__ __forceinline__ uint32_t nv_p_block_scale(float x) {
     return e4m3_encode_sat(ex2_approx(x) * 448.f);
 }
 
+// log2(2688 / v) for a positive E4M3 scale value v (exact in fp32), as two
+// parts whose sum carries one rounding of the fraction: with v = 2^(E - 127) * s,
+// s in [1, 2), 2688 = 2^11 * 1.3125, so log2(2688 / v) = (138 - E) + (log2 1.3125
+// - log2 s).  ei = 138 - E is an exact integer; fr lies in (-0.61, 0.40], so
+// ei + fr (or (ei + 2) / 8 + fr / 8) rounds once at the size of the result.
+// lg2 runs only on the significand.  v = 0 gives meaningless parts; callers
+// select on the scale code.
+__device__ __forceinline__ void nv_p_scale_log2_parts(float v, float& ei, float& fr) {
+    const uint32_t bits = __float_as_uint(v);
+    fr = 0.39231742277876f - lg2_approx(__uint_as_float((bits & 0x7FFFFFu) | 0x3F800000u));
+    ei = static_cast<float>(138 - static_cast<int>(bits >> 23));
+}
+
 // Block exponent from the bfloat16 bit pattern of a block maximum (>= 0)
 // under a scale boundary Qmax in (4, 8]: the smallest e with amax <= Qmax * 2^e
 // is floor(log2 amax) - 2, plus one when the significand exceeds Qmax / 4,
