@@ -208,7 +208,9 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
     constexpr int S = C::kStages;
     constexpr int NT = C::kTiles;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // Aligned by an offset from the shared array itself, so every derived pointer
+    // keeps the shared address space (32-bit addressing, nothing held as a generic pointer).
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
     uint8_t* sQ = smem + C::kOffQ;
     uint8_t* sK = smem + C::kOffK;

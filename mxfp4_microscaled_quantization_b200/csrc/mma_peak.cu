@@ -37,7 +37,9 @@ __device__ __forceinline__ uint64_t atom_desc(const void* p) {
 __global__ void __launch_bounds__(kThreads) mxf4_mma_loop_kernel(int iters, uint32_t* status,
                                                                   unsigned long long* cycles) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // Aligned by an offset from the shared array itself, so every derived pointer
+    // keeps the shared address space (32-bit addressing, nothing held as a generic pointer).
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sA = smem;           // 128 rows x 64 bytes (K = 128 E2M1 values), 64-byte swizzle
     uint8_t* sB = smem + 8192;    // the same for B
     uint8_t* sSf = smem + 16384;  // scale atoms of A and B (512 bytes each)
