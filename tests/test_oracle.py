@@ -3,8 +3,9 @@ the mathematics fix (no GPU).
 
 Source: "MXAttention: Data-Free Optimal Scaling and Pre-Normalization
 Quantization for MXFP4 Attention", abstract: MXFP4 (OCP MX) operands, the UOS
-boundary Qmax = 7.25, PNQ ("quantizes unnormalized softmax exponentials
-before row-wise summation to preserve normalization by construction").
+boundary Qmax = 7.25, and PNQ (the exponentials exp(s - m) are quantized before
+the row sum, so the sum is built from the same values that weight V and the
+normalization holds by construction).
 
 Each check is independent of the oracle's own code: brute-force argmin for the
 rounding, closed forms on the bit patterns for the scale rules, numpy's direct
@@ -240,9 +241,9 @@ def test_quantize_rows_layout_hand_case():
 
 @pytest.mark.parametrize("rule", ["ocp", "uos"])
 def test_quantize_equivariance_power_of_two(rule):
-    """'Distribution-independent' (abstract): the scale depends only on the block maximum,
-    so scaling a block by 2^k leaves the codes unchanged and shifts e by k; negation flips
-    only the sign bits."""
+    """The abstract presents UOS as needing no calibration data: the scale depends only on
+    the block maximum, so scaling a block by 2^k leaves the codes unchanged and shifts e by
+    k; negation flips only the sign bits."""
     rng = np.random.default_rng(2)
     x = rng.standard_normal((64, 128)).astype(np.float32)
     c0, s0 = oracle.quantize_rows(_bits(x), rule)
