@@ -17,9 +17,10 @@
 //                      TMEM lane): running max, per-32-column block exponent
 //                      (UOS/OCP) in the log domain, the exponentials with the
 //                      block scale folded into the bias of one FMA -- under
-//                      PNQ 8 of 16 pairs on the MUFU and 8 on the FMA pipe (a
-//                      code-only stand-in for 2^w), without PNQ 10 and 6 (a
-//                      full polynomial exponential) -- E2M1 packing of P into
+//                      PNQ 9 of 16 pairs on the MUFU and 7 on the FMA pipe (a
+//                      code-only stand-in for 2^w; NVFP4 8 and 8), without
+//                      PNQ 10 and 6 (a full polynomial exponential) -- E2M1
+//                      packing of P into
 //                      shared memory, O rescale in TMEM when the max moved,
 //                      and the final O / l.
 //   warp 8 (one lane)  TMA producer: both Q tiles + scales once, then K and
@@ -111,11 +112,12 @@ struct Cfg {
     static constexpr int kSfSlots = NV ? 2 : kStages;
     static constexpr int kOCols = D + 16;
     // Of the 16 exponential pairs of a 32-column block, this many go to the FMA
-    // pipe instead of the MUFU: 8 with PNQ (the code-only stand-in for 2^w,
-    // exp2_code_sat_x2), 6 without (the full polynomial, exp2_fma_x2); pair q is
-    // one of them when (q * n) mod 16 < n, which spreads them evenly.
+    // pipe instead of the MUFU: with PNQ (the code-only stand-in for 2^w,
+    // exp2_code_sat_x2) 7 for MXFP4 and 8 for NVFP4, whose block scales add MUFU
+    // work of their own; 6 without PNQ (the full polynomial, exp2_fma_x2).  Pair q
+    // is one of them when (q * n) mod 16 < n, which spreads them evenly.
     __host__ __device__ static constexpr bool fma_pair(int q, bool pnq) {
-        const int n = pnq ? 8 : 6;  // measured best for both formats
+        const int n = pnq ? (NV ? 8 : 7) : 6;  // measured best for each format
         return (q * n) % 16 < n;
     }
 
