@@ -339,10 +339,10 @@ def long_video_leg(torch, mx, steps=3):
             "step_tflops": w.flops / (step / 1e3) / 1e12, "steps": steps}
 
 
-# MUFU exponentials per S element in mxattn_fwd_kernel with PNQ: 8 of every 16
-# pairs on the MUFU (ex2.approx), 8 on the FMA pipe; plus the rescale factor,
-# one per row and 128-column key tile.  Block exponents take no exponential.
-MUFU_EX2_PER_ELEMENT = 8.0 / 16 + 1.0 / 128
+# MUFU exponentials per S element in mxattn_fwd_kernel with MXFP4 and PNQ: 9 of
+# every 16 pairs on the MUFU (ex2.approx), 7 on the FMA pipe; plus the rescale
+# factor, one per row and 128-column key tile.  Block exponents take no exponential.
+MUFU_EX2_PER_ELEMENT = 9.0 / 16 + 1.0 / 128
 
 
 def mufu_roofline(w, attn_ms, clocks, sms=148, ex2_per_clk_per_sm=16):
