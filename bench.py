@@ -674,7 +674,9 @@ def run_gpu(args, rank, world, local_rank):
             "mufu_roofline": mufu_roofline(w, attn_avg_ms, clocks),
             "uos_pnq_overhead": overhead,
             "nvfp4": nvfp4,
-            "gpu_launches": (4 if nv_step else 3) * args.steps,
+            # per step: MXFP4 prepare (one fused quantize launch) + attention; NVFP4 prepare is
+            # the amax pass and two quantizers, then attention
+            "gpu_launches": (4 if nv_step else 2) * args.steps,
             "clocks": clocks,
             "quantize_sweep": quant,
             "long_video_dit": long_leg,

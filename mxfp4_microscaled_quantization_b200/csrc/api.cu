@@ -115,11 +115,8 @@ MXATTN_API mxattn_status mxattn_quantize_qmax(const void* x, int64_t rows, int64
     if (x == nullptr || codes == nullptr || scales == nullptr) return MXATTN_ERR_INVALID;
     if (!aligned(x, 16) || !aligned(codes, 4)) return MXATTN_ERR_INVALID;
     if (rows > (int64_t(1) << 40) / cols) return MXATTN_ERR_UNSUPPORTED;
-    const void* xs[1] = {x};
-    uint8_t* cs[1] = {codes};
-    uint8_t* ss[1] = {scales};
-    cudaError_t e = mxattn::launch_quantize_rows(xs, cs, ss, 1, rows, static_cast<int>(cols), th.bf16, 0, 1, 1, 1,
-                                                 nullptr, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = mxattn::launch_quantize_rows(x, codes, scales, rows, static_cast<int>(cols), th.bf16, nullptr,
+                                                 reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
 }
 
@@ -139,9 +136,8 @@ MXATTN_API mxattn_status mxattn_quantize_vt(const void* v, int64_t BH, int64_t N
     if (d != 64 && d != 128) return MXATTN_ERR_UNSUPPORTED;
     if (N > kMaxN || BH > 65535) return MXATTN_ERR_UNSUPPORTED;
     if (!aligned(v, 16) || !aligned(codes_t, 16)) return MXATTN_ERR_INVALID;
-    const int G = static_cast<int>((N + 127) / 128);
-    cudaError_t e = mxattn::launch_quantize_vt(v, BH, static_cast<int>(N), static_cast<int>(d), th.bf16, 0,
-                                               G, codes_t, scales_t, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = mxattn::launch_quantize_vt(v, BH, static_cast<int>(N), static_cast<int>(d), th.bf16, codes_t,
+                                               scales_t, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
 }
 
@@ -161,18 +157,13 @@ MXATTN_API mxattn_status mxattn_prepare_qmax(const void* Q, const void* K, const
     if (st != MXATTN_OK) return st;
     if (Q == nullptr || K == nullptr || V == nullptr) return MXATTN_ERR_INVALID;
     if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16)) return MXATTN_ERR_INVALID;
-    if (static_cast<int64_t>(B) * H > 65535) return MXATTN_ERR_UNSUPPORTED;  // grid.y of the V^T quantizer
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
     const int64_t BH = static_cast<int64_t>(B) * H;
     const int G = (N + 127) / 128;
-    const void* xs[2] = {Q, K};
-    uint8_t* cs[2] = {ws + L.q_codes, ws + L.k_codes};
-    uint8_t* ss[2] = {ws + L.q_sf, ws + L.k_sf};
-    cudaError_t e = mxattn::launch_quantize_rows(xs, cs, ss, 2, BH * N, d, th.bf16, 1, N, G, BH, status, s);
-    if (e != cudaSuccess) return MXATTN_ERR_CUDA;
-    e = mxattn::launch_quantize_vt(V, BH, N, d, th.bf16, 1, G, ws + L.vt_codes, ws + L.v_sf, s);
+    cudaError_t e = mxattn::launch_prepare(Q, K, V, BH, N, d, th.bf16, G, ws + L.q_codes, ws + L.k_codes,
+                                           ws + L.vt_codes, ws + L.q_sf, ws + L.k_sf, ws + L.v_sf, status, s);
     return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA;
 }
 

@@ -669,22 +669,10 @@ __global__ void __launch_bounds__(Cfg<D, T, NV>::kThreads, 1)
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q{};
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
 // 3-D byte tensor [outer, rows, inner_bytes] with a (box_inner x box_rows x 1) box.
 bool encode_map(CUtensorMap* map, const void* base, uint64_t inner_bytes, uint64_t rows, uint64_t outer,
                 uint32_t box_inner, uint32_t box_rows) {
-    auto fn = get_encode_fn();
+    auto fn = tensor_map_encoder();
     if (fn == nullptr) return false;
     cuuint64_t dims[3] = {inner_bytes, rows, outer};
     cuuint64_t strides[2] = {inner_bytes, inner_bytes * rows};

@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
 
@@ -19,18 +20,25 @@ constexpr int64_t kMaxAttentionN = int64_t(1) << 24;
 // N <= kMaxAttentionN and the grid size (UNSUPPORTED).
 mxattn_status check_attention_shape(int B, int H, int N, int d, int kv_tile, int pnq, const float* O);
 
-// Row quantization of `ntensors` (1 or 2) bf16 tensors of shape [rows, cols].
-// regroup = 0: row-major scales; regroup = 1: rows are (bh, r < N), scales in
-// the 128-row regrouped order (padding rows zeroed).  Clears *status when
-// status != nullptr.
-cudaError_t launch_quantize_rows(const void* const* x, uint8_t* const* codes, uint8_t* const* scales, int ntensors,
-                                 int64_t rows, int cols, uint32_t sf_thresh, int regroup, int N, int groups, int64_t BH,
-                                 uint32_t* status, cudaStream_t stream);
+// Row quantization of a bf16 tensor [rows, cols] (cols a multiple of 32) with
+// row-major scales [rows, cols/32].  Clears *status when status != nullptr.
+cudaError_t launch_quantize_rows(const void* x, uint8_t* codes, uint8_t* scales, int64_t rows, int cols,
+                                 uint32_t sf_thresh, uint32_t* status, cudaStream_t stream);
 
-// V [BH, N, d] -> V^T codes [BH, d, Npad/2] and scales (row-major
-// [BH, d, Npad/32] when regroup = 0, regrouped per 128 tokens when 1).
-cudaError_t launch_quantize_vt(const void* v, int64_t BH, int N, int d, uint32_t sf_thresh, int regroup, int groups,
-                               uint8_t* codes_t, uint8_t* scales_t, cudaStream_t stream);
+// V [BH, N, d] -> V^T codes [BH, d, Npad/2] and row-major scales [BH, d, Npad/32].
+cudaError_t launch_quantize_vt(const void* v, int64_t BH, int N, int d, uint32_t sf_thresh, uint8_t* codes_t,
+                               uint8_t* scales_t, cudaStream_t stream);
+
+// The forward's operand preparation in one persistent launch: Q and K [BH, N,
+// d] bf16 -> codes [BH, N, d/2] + regrouped scales, V -> V^T codes [BH, d,
+// Npad/2] + regrouped scales (channel rows d..127 of each group at scale 2^0).
+// Clears *status.  Q, K, V 16-byte aligned.
+cudaError_t launch_prepare(const void* Q, const void* K, const void* V, int64_t BH, int N, int d, uint32_t sf_thresh,
+                           int groups, uint8_t* q_codes, uint8_t* k_codes, uint8_t* vt_codes, uint8_t* q_sf,
+                           uint8_t* k_sf, uint8_t* v_sf, uint32_t* status, cudaStream_t stream);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (nullptr if unavailable).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // Row-major Q/K/V^T scales -> regrouped scales; clears *status.
 cudaError_t launch_regroup_sf(const uint8_t* q_scales, const uint8_t* k_scales, const uint8_t* vt_scales, int64_t BH,

@@ -5,20 +5,20 @@
 // power-of-two microscaling; scale rule OCP (floor(log2 amax) - 2) or UOS
 // (smallest e with amax <= Qmax * 2^e, Qmax = 7.25).
 //
-//  * quantize_rows_kernel: blocks of 32 consecutive elements of a row (Q, K,
-//    and the standalone op).  Each thread loads 16 bytes (8 bf16), a quad of
+//  * quantize_rows_kernel: blocks of 32 consecutive elements of a row (the
+//    standalone op).  Each thread loads 16 bytes (8 bf16), a quad of
 //    lanes owns one block: the block maximum is an integer max over |bf16|
 //    bit patterns plus two xor-shuffles, the exponent comes from the maximum's
 //    exponent and mantissa fields, the 8 scaled values go through four
 //    cvt.rn.satfinite.e2m1x2 and leave as one 32-bit store.  The quad's first
-//    lane stores the E8M0 byte (row-major, or regrouped per 128 rows in the
-//    order the tensor core reads scale factors).
+//    lane stores the E8M0 byte (row-major scales).
 //  * quantize_vt_kernel: V blocks of 32 consecutive tokens per channel,
 //    written transposed (V^T, tokens contiguous): a CTA stages 128 tokens x d
 //    channels in shared memory and each thread quantizes the blocks of a pair
 //    of channels over a run of tokens from there (one 32-bit shared-memory
-//    read per token for both channels).
+//    read per token for both channels), row-major scales.
 //  * regroup_sf_kernel: row-major scales -> the 128-row regrouped order.
+// The forward's own preparation (regrouped scales, one launch) is prepare.cu.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -64,19 +64,12 @@ __device__ __forceinline__ uint32_t quantize_quad(uint4 raw, uint32_t sf_thresh,
     return pack_e2m1x8(f);
 }
 
-struct RowsArgs {
-    const uint16_t* x[2];
-    uint8_t* codes[2];
-    uint8_t* scales[2];
-};
-
 // Row quantization with row-major scales [rows, cols/32] (the standalone op):
 // grid-stride over 16-byte chunks, kUnroll loads in flight per lane.
-__global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(RowsArgs a, int64_t n_chunks, int cols, uint32_t sf_thresh,
-                                                                      uint32_t* status) {
-    const uint16_t* __restrict__ x = a.x[0];
-    uint32_t* __restrict__ codes = reinterpret_cast<uint32_t*>(a.codes[0]);
-    uint8_t* __restrict__ scales = a.scales[0];
+__global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const uint16_t* __restrict__ x,
+                                                                      uint32_t* __restrict__ codes,
+                                                                      uint8_t* __restrict__ scales, int64_t n_chunks,
+                                                                      uint32_t sf_thresh, uint32_t* status) {
     if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0u;
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x) >> 5;
@@ -101,51 +94,6 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(RowsArgs a
     }
 }
 
-// Forward's Q/K quantization: one CTA per (128-row group, bh, tensor).  Rows
-// past N are zeros; the group's 512 scale bytes are assembled in shared memory
-// in the regrouped order and written out contiguously.
-template <int D>
-__global__ void __launch_bounds__(kQuantThreads) quantize_rows_grouped_kernel(RowsArgs a, int N, int groups, uint32_t sf_thresh,
-                                                                              uint32_t* status) {
-    constexpr int kChunksPerRow = D / 8;                          // 16-byte chunks per row
-    constexpr int kPerThread = 128 * kChunksPerRow / kQuantThreads;
-    __shared__ __align__(16) uint8_t sf[512];
-    const uint16_t* __restrict__ x = blockIdx.z ? a.x[1] : a.x[0];
-    uint32_t* __restrict__ codes = reinterpret_cast<uint32_t*>(blockIdx.z ? a.codes[1] : a.codes[0]);
-    uint8_t* __restrict__ scales = blockIdx.z ? a.scales[1] : a.scales[0];
-    const int g = blockIdx.x;
-    const int64_t bh = blockIdx.y;
-    if (status != nullptr && g == 0 && bh == 0 && blockIdx.z == 0 && threadIdx.x == 0) *status = 0u;
-    reinterpret_cast<uint32_t*>(sf)[threadIdx.x & 127] = 0u;
-    const int64_t row0 = bh * N + static_cast<int64_t>(g) * 128;  // global row of the group's first row
-    const int rows_valid = min(128, N - g * 128);
-    uint4 raw[kPerThread];
-#pragma unroll
-    for (int u = 0; u < kPerThread; ++u) {
-        const int c = threadIdx.x + u * kQuantThreads;
-        const int m = c / kChunksPerRow;
-        raw[u] = (m < rows_valid) ? __ldcs(reinterpret_cast<const uint4*>(x + (row0 + m) * D) + (c % kChunksPerRow))
-                                  : make_uint4(0, 0, 0, 0);
-    }
-    __syncthreads();  // sf cleared
-#pragma unroll
-    for (int u = 0; u < kPerThread; ++u) {
-        const int c = threadIdx.x + u * kQuantThreads;
-        const int m = c / kChunksPerRow;
-        int e;
-        const uint32_t packed = quantize_quad(raw[u], sf_thresh, e);
-        if (m < rows_valid) codes[(row0 + m) * (D / 8) + (c % kChunksPerRow)] = packed;
-        if ((threadIdx.x & 3) == 0) {
-            const int k = (c % kChunksPerRow) / 4;
-            sf[(m & 31) * 16 + (m >> 5) * 4 + k] = static_cast<uint8_t>(e + 127);  // zero rows give e = -127
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x < 32)
-        reinterpret_cast<uint4*>(scales + (bh * groups + g) * 512)[threadIdx.x] =
-            reinterpret_cast<const uint4*>(sf)[threadIdx.x];
-}
-
 // V^T quantization: grid (G token groups of 128, BH), 128 threads.  The CTA
 // stages 128 tokens x D channels (bf16) in shared memory.  Each thread then
 // owns a pair of adjacent channels over a run of 256 / D * 16 tokens (64 for
@@ -155,8 +103,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_grouped_kernel(Ro
 // as contiguous 16-byte stores.
 template <int D>
 __global__ void __launch_bounds__(128) quantize_vt_kernel(const uint16_t* __restrict__ v, int N, int npad, uint32_t sf_thresh,
-                                                          int regroup, int groups, uint8_t* __restrict__ codes_t,
-                                                          uint8_t* __restrict__ scales_t) {
+                                                          uint8_t* __restrict__ codes_t, uint8_t* __restrict__ scales_t) {
     constexpr int kPairs = D / 2;             // channel pairs
     constexpr int kRuns = 128 / kPairs;       // token runs per 128-token group (2 or 4)
     constexpr int kRun = 128 / kRuns;         // tokens per run (64 or 32)
@@ -182,7 +129,6 @@ __global__ void __launch_bounds__(128) quantize_vt_kernel(const uint16_t* __rest
     const int cp = tid % kPairs;   // channels 2 cp, 2 cp + 1
     const int run = tid / kPairs;  // tokens [run * kRun, run * kRun + kRun) of the group
     const uint32_t* tile32 = reinterpret_cast<const uint32_t*>(tile);
-    uint32_t sfbytes[2] = {0u, 0u};  // per channel: the scale bytes of this run's blocks
 #pragma unroll
     for (int b = 0; b < kBlocks; ++b) {
         uint32_t raw[32];  // token i of the block: channel 2 cp in the low half, 2 cp + 1 in the high half
@@ -209,32 +155,9 @@ __global__ void __launch_bounds__(128) quantize_vt_kernel(const uint16_t* __rest
             }
             const int ch = 2 * cp + h;
             uint8_t* rowp = codes_t + (bh * D + ch) * static_cast<int64_t>(npad / 2);
-            if (tb < npad) *reinterpret_cast<uint4*>(rowp + tb / 2) = make_uint4(words[0], words[1], words[2], words[3]);
-            const uint32_t sbyte = static_cast<uint32_t>(e + 127);
-            sfbytes[h] |= sbyte << (8 * b);
-            if (!regroup && tb < npad) scales_t[(bh * D + ch) * static_cast<int64_t>(npad / 32) + tb / 32] = sbyte;
-        }
-    }
-    if (regroup) {
-        // group g of 128 tokens; channel ch plays the role of the row, block k of the
-        // group its byte k: this run's blocks are bytes run * kBlocks ...
-        uint8_t* grp = scales_t + (bh * groups + g) * 512;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int ch = 2 * cp + h;
-            uint8_t* word = grp + (ch & 31) * 16 + (ch >> 5) * 4 + run * kBlocks;
-            if constexpr (kBlocks == 2)
-                *reinterpret_cast<uint16_t*>(word) = static_cast<uint16_t>(sfbytes[h]);
-            else
-                *word = static_cast<uint8_t>(sfbytes[h]);
-        }
-        if (D < 128 && run == 0) {
-            // channel rows D..127 of the group: scale 2^0, so the extra ones-row the
-            // attention kernel appends to V^T (row D) is read with unit scale
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int c2 = 2 * cp + h + D;
-                *reinterpret_cast<uint32_t*>(grp + (c2 & 31) * 16 + (c2 >> 5) * 4) = 0x7F7F7F7Fu;
+            if (tb < npad) {
+                *reinterpret_cast<uint4*>(rowp + tb / 2) = make_uint4(words[0], words[1], words[2], words[3]);
+                scales_t[(bh * D + ch) * static_cast<int64_t>(npad / 32) + tb / 32] = static_cast<uint8_t>(e + 127);
             }
         }
     }
@@ -288,39 +211,24 @@ int grid_for(int64_t work_items, int per_block) {
 
 }  // namespace
 
-cudaError_t launch_quantize_rows(const void* const* x, uint8_t* const* codes, uint8_t* const* scales, int ntensors,
-                                 int64_t rows, int cols, uint32_t sf_thresh, int regroup, int N, int groups, int64_t BH,
-                                 uint32_t* status, cudaStream_t stream) {
-    RowsArgs a{};
-    for (int t = 0; t < ntensors; ++t) {
-        a.x[t] = static_cast<const uint16_t*>(x[t]);
-        a.codes[t] = codes[t];
-        a.scales[t] = scales[t];
-    }
-    if (regroup) {
-        dim3 grid(groups, static_cast<unsigned>(BH), ntensors);
-        if (cols == 128)
-            quantize_rows_grouped_kernel<128><<<grid, kQuantThreads, 0, stream>>>(a, N, groups, sf_thresh, status);
-        else
-            quantize_rows_grouped_kernel<64><<<grid, kQuantThreads, 0, stream>>>(a, N, groups, sf_thresh, status);
-        return cudaGetLastError();
-    }
+cudaError_t launch_quantize_rows(const void* x, uint8_t* codes, uint8_t* scales, int64_t rows, int cols,
+                                 uint32_t sf_thresh, uint32_t* status, cudaStream_t stream) {
     const int64_t n_chunks = rows * cols / 8;
-    dim3 grid(grid_for(n_chunks / kUnroll, kQuantThreads), ntensors);
-    quantize_rows_kernel<<<grid, kQuantThreads, 0, stream>>>(a, n_chunks, cols, sf_thresh, status);
+    quantize_rows_kernel<<<grid_for(n_chunks / kUnroll, kQuantThreads), kQuantThreads, 0, stream>>>(
+        static_cast<const uint16_t*>(x), reinterpret_cast<uint32_t*>(codes), scales, n_chunks, sf_thresh, status);
     return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_vt(const void* v, int64_t BH, int N, int d, uint32_t sf_thresh, int regroup, int groups,
-                               uint8_t* codes_t, uint8_t* scales_t, cudaStream_t stream) {
+cudaError_t launch_quantize_vt(const void* v, int64_t BH, int N, int d, uint32_t sf_thresh, uint8_t* codes_t,
+                               uint8_t* scales_t, cudaStream_t stream) {
     const int npad = (N + 31) / 32 * 32;
-    dim3 grid(groups, static_cast<unsigned>(BH));
+    dim3 grid((N + 127) / 128, static_cast<unsigned>(BH));
     if (d == 128)
-        quantize_vt_kernel<128><<<grid, 128, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, sf_thresh, regroup,
-                                                           groups, codes_t, scales_t);
+        quantize_vt_kernel<128><<<grid, 128, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, sf_thresh, codes_t,
+                                                           scales_t);
     else
-        quantize_vt_kernel<64><<<grid, 128, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, sf_thresh, regroup,
-                                                          groups, codes_t, scales_t);
+        quantize_vt_kernel<64><<<grid, 128, 0, stream>>>(static_cast<const uint16_t*>(v), N, npad, sf_thresh, codes_t,
+                                                          scales_t);
     return cudaGetLastError();
 }
 
