@@ -131,6 +131,19 @@ def test_ragged_shapes(N, d, T):
     check_codes(ws, Q, K, V, "ocp")
 
 
+def test_more_heads_than_a_grid_dimension():
+    """B*H above 65,535 (one fused preparation launch, one attention CTA per head and
+    tile pair): sampled heads, including both sides of 65,536, against the oracle."""
+    B, H, N, d, T = 1, 66000, 3, 64, 64
+    Q, K, V = wl.gaussian_qkv(B, H, N, d, seed=66)
+    O, ws = run_forward(Q, K, V, T, True, "uos")
+    heads = [0, 1, 4097, 65534, 65535, 65536, 65537, H - 1]
+    check_codes(ws, Q, K, V, "uos", heads=heads)
+    sel = lambda X: X[:, heads]
+    R = oracle.attention(sel(Q), sel(K), sel(V), T, rule="uos", pnq=True)
+    assert_close(O[:, heads], R, "B*H = 66000, sampled heads")
+
+
 def test_explicit_softmax_scale():
     Q, K, V = wl.gaussian_qkv(1, 2, 300, 64, seed=11)
     O, _ = run_forward(Q, K, V, 64, True, "uos", scale=0.3)
