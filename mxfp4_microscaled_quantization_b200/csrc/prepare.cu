@@ -6,7 +6,8 @@
 // Quantization for MXFP4 Attention", abstract -- MXFP4 operands with
 // power-of-two microscaling; scale rule OCP (floor(log2 amax) - 2) or UOS
 // (smallest e with amax <= Qmax * 2^e, Qmax = 7.25).  The arithmetic per block
-// is the one of quantize.cu (quantize_quad and the V^T block loop).
+// is shared with the standalone quantizers (quantize_quad_bf16 and
+// quantize_vt_block_bf16 in ptx.cuh).
 //
 // The work is a list of tiles of 128 tokens x d channels of bf16 (32 KB for
 // d = 128): for every (b, h) and 128-token group, its Q, K and V tile, in that
@@ -58,12 +59,16 @@ namespace {
 
 constexpr uint64_t kPrepTimeoutNs = 2000000000ull;  // 2 s per wait
 constexpr uint32_t kPrepTimeoutCode = 4u;           // MXATTN_ERR_TIMEOUT
-
-template <int D>
-struct PrepCfg {
+// Ring slots per CTA and CTAs per SM (measured best: two slots, three CTAs).
 #ifndef MXATTN_PREP_STAGES
 #define MXATTN_PREP_STAGES 2
 #endif
+#ifndef MXATTN_PREP_CTAS
+#define MXATTN_PREP_CTAS 3
+#endif
+
+template <int D>
+struct PrepCfg {
     static constexpr int kStages = MXATTN_PREP_STAGES;
     static constexpr int kTileBytes = 128 * D * 2;
     static constexpr int kConsumers = 2 * D;             // 256 (d = 128) or 128 (d = 64)
@@ -94,34 +99,7 @@ struct PrepArgs {
     uint32_t sf_thresh;
 };
 
-// One 32-element block spread over a quad of lanes (8 elements each): packed
-// codes of this lane's elements, the block exponent in e_out.
-__device__ __forceinline__ uint32_t quantize_quad8(uint4 raw, uint32_t sf_thresh, int& e_out) {
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-    uint32_t amax = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        amax = max(amax, w[i] & 0x7FFFu);
-        amax = max(amax, (w[i] >> 16) & 0x7FFFu);
-    }
-    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    const int e = block_exponent_bf16(amax, sf_thresh);
-    const float sc = exp2_neg_int(e);
-    float f[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16) * sc;
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u) * sc;
-    }
-    e_out = e;
-    return pack_e2m1x8(f);
-}
-
 template <int D>
-#ifndef MXATTN_PREP_CTAS
-#define MXATTN_PREP_CTAS 3
-#endif
 __global__ void __launch_bounds__(PrepCfg<D>::kThreads, MXATTN_PREP_CTAS)
     prepare_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrepArgs p) {
@@ -208,7 +186,7 @@ __global__ void __launch_bounds__(PrepCfg<D>::kThreads, MXATTN_PREP_CTAS)
                 const int m = c / C::kChunksPerRow;
                 const int cc = c % C::kChunksPerRow;
                 int e;
-                const uint32_t packed = quantize_quad8(raw[u], p.sf_thresh, e);
+                const uint32_t packed = quantize_quad_bf16(raw[u], p.sf_thresh, e);
                 if (t0 + m < p.N) codes[(bh * p.N + t0 + m) * (D / 8) + cc] = packed;
                 // row m's scale word: byte k for its block k (rows past N: zero data, byte 0)
                 uint8_t* word = grp + (m & 31) * 16 + (m >> 5) * 4;
@@ -222,35 +200,22 @@ __global__ void __launch_bounds__(PrepCfg<D>::kThreads, MXATTN_PREP_CTAS)
             const int run = tid / C::kPairs;
             const uint32_t* tile32 = reinterpret_cast<const uint32_t*>(t8);
             uint32_t raw[32];
-            uint32_t amax0 = 0, amax1 = 0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                raw[i] = tile32[(run * 32 + i) * C::kPairs + cp];
-                amax0 = max(amax0, raw[i] & 0x7FFFu);
-                amax1 = max(amax1, (raw[i] >> 16) & 0x7FFFu);
-            }
+            for (int i = 0; i < 32; ++i) raw[i] = tile32[(run * 32 + i) * C::kPairs + cp];
             mbar_arrive(bar_empty + s);
+            uint32_t words[2][4];
+            int e[2];
+            quantize_vt_block_bf16(raw, p.sf_thresh, words, e);
             const int tb = t0 + run * 32;  // first token of the block
             uint8_t* grp = p.v_sf + bg * 512;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const int e = block_exponent_bf16(h ? amax1 : amax0, p.sf_thresh);
-                const float sc = exp2_neg_int(e);
-                uint32_t words[4];
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    float f[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        f[i] = __uint_as_float(h ? (raw[8 * w + i] & 0xFFFF0000u) : (raw[8 * w + i] << 16)) * sc;
-                    words[w] = pack_e2m1x8(f);
-                }
                 const int ch = 2 * cp + h;
                 if (tb < p.npad)
                     *reinterpret_cast<uint4*>(p.vt_codes + (bh * D + ch) * static_cast<int64_t>(p.npad / 2) + tb / 2) =
-                        make_uint4(words[0], words[1], words[2], words[3]);
+                        make_uint4(words[h][0], words[h][1], words[h][2], words[h][3]);
                 // channel ch plays the role of the row, block `run` of the group its byte
-                grp[(ch & 31) * 16 + (ch >> 5) * 4 + run] = static_cast<uint8_t>(e + 127);
+                grp[(ch & 31) * 16 + (ch >> 5) * 4 + run] = static_cast<uint8_t>(e[h] + 127);
             }
             if (D < 128 && run == 0) {
                 // channel rows D..127 of the group: scale 2^0, so the extra ones-row the

@@ -40,30 +40,6 @@ constexpr int kQuantThreads = 256;
 constexpr int kUnroll = MXATTN_QUANT_UNROLL;             // 16-byte loads in flight per lane
 constexpr int kCtasPerSm = MXATTN_QUANT_CTAS_PER_SM;     // grid of the grid-stride quantizer
 
-// One 32-element block spread over a quad of lanes (8 elements each).
-// Returns the packed codes of this lane's 8 elements; `e_out` gets the block exponent.
-__device__ __forceinline__ uint32_t quantize_quad(uint4 raw, uint32_t sf_thresh, int& e_out) {
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-    uint32_t amax = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        amax = max(amax, w[i] & 0x7FFFu);
-        amax = max(amax, (w[i] >> 16) & 0x7FFFu);
-    }
-    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    const int e = block_exponent_bf16(amax, sf_thresh);
-    const float sc = exp2_neg_int(e);
-    float f[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16) * sc;
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u) * sc;
-    }
-    e_out = e;
-    return pack_e2m1x8(f);
-}
-
 // Row quantization with row-major scales [rows, cols/32] (the standalone op):
 // grid-stride over 16-byte chunks, kUnroll loads in flight per lane.
 __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const uint16_t* __restrict__ x,
@@ -85,7 +61,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_rows_kernel(const uint
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t i = base + u * 32 + lane;
             int e;
-            const uint32_t packed = quantize_quad(raw[u], sf_thresh, e);
+            const uint32_t packed = quantize_quad_bf16(raw[u], sf_thresh, e);
             if (i < n_chunks) {
                 codes[i] = packed;
                 if ((lane & 3) == 0) scales[i >> 2] = static_cast<uint8_t>(e + 127);
@@ -132,32 +108,19 @@ __global__ void __launch_bounds__(128) quantize_vt_kernel(const uint16_t* __rest
 #pragma unroll
     for (int b = 0; b < kBlocks; ++b) {
         uint32_t raw[32];  // token i of the block: channel 2 cp in the low half, 2 cp + 1 in the high half
-        uint32_t amax0 = 0, amax1 = 0;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            raw[i] = tile32[(run * kRun + 32 * b + i) * kPairs + cp];
-            amax0 = max(amax0, raw[i] & 0x7FFFu);
-            amax1 = max(amax1, (raw[i] >> 16) & 0x7FFFu);
-        }
+        for (int i = 0; i < 32; ++i) raw[i] = tile32[(run * kRun + 32 * b + i) * kPairs + cp];
+        uint32_t words[2][4];
+        int e[2];
+        quantize_vt_block_bf16(raw, sf_thresh, words, e);
         const int tb = t0 + run * kRun + 32 * b;  // first token of the block
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const int e = block_exponent_bf16(h ? amax1 : amax0, sf_thresh);
-            const float sc = exp2_neg_int(e);
-            uint32_t words[4];
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                float f[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    f[i] = __uint_as_float(h ? (raw[8 * w + i] & 0xFFFF0000u) : (raw[8 * w + i] << 16)) * sc;
-                words[w] = pack_e2m1x8(f);
-            }
             const int ch = 2 * cp + h;
             uint8_t* rowp = codes_t + (bh * D + ch) * static_cast<int64_t>(npad / 2);
             if (tb < npad) {
-                *reinterpret_cast<uint4*>(rowp + tb / 2) = make_uint4(words[0], words[1], words[2], words[3]);
-                scales_t[(bh * D + ch) * static_cast<int64_t>(npad / 32) + tb / 32] = static_cast<uint8_t>(e + 127);
+                *reinterpret_cast<uint4*>(rowp + tb / 2) = make_uint4(words[h][0], words[h][1], words[h][2], words[h][3]);
+                scales_t[(bh * D + ch) * static_cast<int64_t>(npad / 32) + tb / 32] = static_cast<uint8_t>(e[h] + 127);
             }
         }
     }
