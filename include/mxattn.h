@@ -126,10 +126,10 @@ size_t mxattn_workspace_size(int B, int H, int N, int d);
  *   d in {64, 128}; kv_tile in {64, 128}; 1 <= N <= 2^24; pnq in {0, 1};
  *   rule applies to Q, K, V and P; softmax_scale <= 0 selects 1/sqrt(d).
  *   workspace: >= mxattn_workspace_size(B, H, N, d) bytes, 256-byte aligned.
- * Launches three kernels on `stream`: Q/K quantize, V^T quantize, attention.
- * The attention kernel's waits are bounded; if one gives up it records
- * MXATTN_ERR_TIMEOUT in the workspace status word (see
- * mxattn_workspace_status) and O is unspecified.
+ * Launches two kernels on `stream`: the operand preparation (Q, K and V^T
+ * quantized in one launch) and the attention.  Both kernels' waits are
+ * bounded; if one gives up it records MXATTN_ERR_TIMEOUT in the workspace
+ * status word (see mxattn_workspace_status) and O is unspecified.
  */
 mxattn_status mxattn_forward(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
                              int kv_tile, int pnq, mxattn_rule rule, float softmax_scale, float* O,
@@ -137,8 +137,9 @@ mxattn_status mxattn_forward(const void* Q, const void* K, const void* V, int B,
 
 /*
  * mxattn_forward in two calls, for callers that time or schedule the steps
- * separately: mxattn_prepare launches the Q/K and V^T quantize kernels into
- * the workspace (and resets its status word); mxattn_attend launches the
+ * separately: mxattn_prepare launches the operand preparation (Q, K and V^T
+ * quantized in one kernel) into the workspace and resets its status word;
+ * mxattn_attend launches the
  * attention kernel on a workspace that mxattn_prepare filled for the same
  * (B, H, N, d) and `rule`.  mxattn_forward == mxattn_prepare + mxattn_attend.
  * Same constraints and errors as mxattn_forward.
