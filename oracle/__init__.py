@@ -11,9 +11,11 @@ Data-Free Optimal Scaling and Pre-Normalization Quantization for MXFP4
 Attention").  Every function here is pinned by the ``-m "not gpu"`` tests
 (E2M1 grid and brute-force rounding, the OCP and UOS scale invariants,
 equivariance, exact online softmax, PNQ normalization, hand-derived golden
-cases; for the NVFP4 comparison variant, torch's float8_e4m3fn conversion,
-brute-force element rounding, equivariance and special cases); none is
-"parity unpinned".
+cases, and two-key-tile cases of the quantized loop with values derived by
+hand, which fail if P is quantized against the tile-local or the final row
+maximum; for the NVFP4 comparison variant, torch's float8_e4m3fn conversion,
+brute-force element rounding, equivariance, special cases and the same
+two-tile cases); none is "parity unpinned".
 """
 from __future__ import annotations
 
