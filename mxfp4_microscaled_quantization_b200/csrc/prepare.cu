@@ -7,7 +7,7 @@
 // power-of-two microscaling; scale rule OCP (floor(log2 amax) - 2) or UOS
 // (smallest e with amax <= Qmax * 2^e, Qmax = 7.25).  The arithmetic per block
 // is shared with the standalone quantizers (quantize_quad_bf16 and
-// quantize_vt_block_bf16 in ptx.cuh).
+// quantize_vt_block_bf16 in mxfp4_block.cuh).
 //
 // The work is a list of tiles of 128 tokens x d channels of bf16 (32 KB for
 // d = 128): for every (b, h) and 128-token group, its Q, K and V tile, in that
@@ -39,6 +39,7 @@
 #include <cstdint>
 
 #include "kernels.cuh"
+#include "mxfp4_block.cuh"
 #include "ptx.cuh"
 
 namespace mxattn {

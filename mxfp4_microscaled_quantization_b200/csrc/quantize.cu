@@ -24,6 +24,7 @@
 #include <cstdint>
 
 #include "kernels.cuh"
+#include "mxfp4_block.cuh"
 #include "ptx.cuh"
 
 namespace mxattn {
