@@ -15,31 +15,40 @@
 
 namespace mxattn {
 
+// Lane-wise maximum of two pairs of unsigned 16-bit values.
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// The block maximum works on |bf16| bit patterns (sign cleared), which order
+// like the magnitudes, two per 32-bit word at a time; the scaling multiplies
+// two fp32 values per instruction by the power of two 2^-e (exact, round to
+// nearest even like the scalar product).
+
 // MXFP4 quantization of one 32-element bf16 block spread over a quad of lanes
-// (lanes 4k .. 4k + 3, 8 elements each in `raw`): the block maximum is an
-// integer max over |bf16| bit patterns plus two xor shuffles, e its block
-// exponent under the scale boundary `mant_thresh`; returns this lane's 8 E2M1
-// codes packed (element 0 in the lowest nibble).  All 32 lanes must call it.
+// (lanes 4k .. 4k + 3, 8 elements each in `raw`): the block maximum is a
+// maximum over |bf16| bit patterns plus two xor shuffles, e its block exponent
+// under the scale boundary `mant_thresh`; returns this lane's 8 E2M1 codes
+// packed (element 0 in the lowest nibble).  All 32 lanes must call it.
 __device__ __forceinline__ uint32_t quantize_quad_bf16(uint4 raw, uint32_t mant_thresh, int& e_out) {
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-    uint32_t amax = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        amax = max(amax, w[i] & 0x7FFFu);
-        amax = max(amax, (w[i] >> 16) & 0x7FFFu);
-    }
+    const uint32_t m2 = vmax_u16x2(vmax_u16x2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu),
+                                   vmax_u16x2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu));
+    uint32_t amax = max(m2 & 0xFFFFu, m2 >> 16);
     amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
     const int e = block_exponent_bf16(amax, mant_thresh);
     const float sc = exp2_neg_int(e);
-    float f[8];
+    uint32_t f[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16) * sc;
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u) * sc;
-    }
+    for (int i = 0; i < 4; ++i) fmul2_bcast(f[2 * i], f[2 * i + 1], w[i] << 16, w[i] & 0xFFFF0000u, sc);
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(f[i]);
     e_out = e;
-    return pack_e2m1x8(f);
+    return pack_e2m1x8(v);
 }
 
 // MXFP4 quantization of two channels over one 32-token block of V: raw[i] holds
@@ -48,23 +57,25 @@ __device__ __forceinline__ uint32_t quantize_quad_bf16(uint4 raw, uint32_t mant_
 // words[h][0]), e[h] its block exponent.
 __device__ __forceinline__ void quantize_vt_block_bf16(const uint32_t (&raw)[32], uint32_t mant_thresh,
                                                        uint32_t (&words)[2][4], int (&e)[2]) {
-    uint32_t amax0 = 0, amax1 = 0;
+    uint32_t m2 = raw[0] & 0x7FFF7FFFu;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        amax0 = max(amax0, raw[i] & 0x7FFFu);
-        amax1 = max(amax1, (raw[i] >> 16) & 0x7FFFu);
-    }
+    for (int i = 1; i < 32; ++i) m2 = vmax_u16x2(m2, raw[i] & 0x7FFF7FFFu);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        e[h] = block_exponent_bf16(h ? amax1 : amax0, mant_thresh);
+        e[h] = block_exponent_bf16(h ? (m2 >> 16) : (m2 & 0xFFFFu), mant_thresh);
         const float sc = exp2_neg_int(e[h]);
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            float f[8];
+            uint32_t f[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                f[i] = __uint_as_float(h ? (raw[8 * w + i] & 0xFFFF0000u) : (raw[8 * w + i] << 16)) * sc;
-            words[h][w] = pack_e2m1x8(f);
+            for (int i = 0; i < 8; i += 2) {
+                const uint32_t a = raw[8 * w + i], b = raw[8 * w + i + 1];
+                fmul2_bcast(f[i], f[i + 1], h ? (a & 0xFFFF0000u) : (a << 16), h ? (b & 0xFFFF0000u) : (b << 16), sc);
+            }
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(f[i]);
+            words[h][w] = pack_e2m1x8(v);
         }
     }
 }
