@@ -100,8 +100,8 @@ MXATTN_API mxattn_status mxattn_forward_noalloc(const void* Q, const void* K, co
     if (need > kNoAllocScratchBytes) return MXATTN_ERR_UNSUPPORTED;  // shape too large for the fixed scratch
     void* scratch = nullptr;
     if (scratch_on_current_device(&scratch) != cudaSuccess) return MXATTN_ERR_CUDA;
-    // The quantize kernels rewrite every workspace byte the attention kernel
-    // reads and reset the status word, so stale contents of the previous call
+    // The preparation kernel rewrites every workspace byte the attention kernel
+    // reads and resets the status word, so stale contents of the previous call
     // do not leak into this one.
     return mxattn_forward(Q, K, V, B, H, N, d, kv_tile, pnq, rule, softmax_scale, O, scratch, kNoAllocScratchBytes,
                           stream);
